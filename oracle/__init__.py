@@ -1,0 +1,29 @@
+"""CPU oracle for multi-head latent attention (MLA): test infrastructure only.
+
+This package is the plain, slow, fp64 statement of what the CUDA path computes.
+Only the test suite, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import it; the product path (the C-ABI library and its Python
+binding) never does, and shares no code with it.
+
+Pinned against what the pages and the mathematics fix (see ``tests/test_oracle_pins.py``):
+the absorb/naive identity, closed forms (one cached row, zero query, two keys),
+library special cases (``scaled_dot_product_attention`` in fp64), brute-force
+top-k masking, the page's parameter counts and cache-size formulas, and planted
+mistakes that must be caught.  Every function here has at least one such pin.
+"""
+
+from .mla_oracle import (  # noqa: F401
+    absorb_q,
+    absorbed_decode,
+    index_mask,
+    latent_attention,
+    mha_cache_bytes,
+    mla_cache_bytes,
+    naive_decode,
+    naive_prefill,
+    out_up,
+    softmax,
+    softmax_scale,
+    split_wkv_b,
+    value_up_params,
+)

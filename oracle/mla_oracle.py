@@ -1,0 +1,240 @@
+"""Plain fp64 CPU statement of multi-head latent attention (MLA), naive and absorbed.
+
+Test infrastructure only: the product path never imports this module (see the package
+docstring).  Every array is upcast to float64 on entry, so bf16 or fp32 inputs are used
+at exactly the values the GPU receives; nothing is rounded in between.
+
+Sources (page title, then section / equation):
+
+* "KV Reconstruction" (DeepSeek-V3 note), "How it works": eqs. (2) and (5),
+  k^C_t = W^UK c^KV_t and v^C_t = W^UV c^KV_t, with W^UK, W^UV in R^{n_h d_h x d_c};
+  the key used by attention is k_{t,i} = [k^C_{t,i}; k^R_t] (192 wide for DeepSeek-V3).
+  Same page, "Naive path": expand, split, concatenate k^R, run ordinary attention.
+  Same page, "Absorb path (default)": the content score equals ((W^UK_i)^T q^C_i)^T c^KV_j
+  and the value mix equals W^UV_i sum_j alpha_j c^KV_j; rotary scores are added separately.
+  Same page, "Official code": the fused wkv_b holds, per head, the d_h key rows first and
+  the d_v value rows after them.
+* "DeepSeek-V3.2-Exp - Absorb key weights", the MQA-decode code excerpt: the query is folded
+  through the first qk_nope_head_dim rows of each head of wkv_b; scores over the cached latent
+  plus scores over the rotary cache, times the softmax scale; an optional -inf mask with 0
+  scattered at the top-k indices; softmax over positions; weighted sum of the cached latent;
+  then the last v_head_dim rows of each head map it back up.
+* "Value up-projection", the MHA-prefill excerpt: wkv_b expansion viewed as
+  [B, S, heads, d_h + d_v], split into k_nope and v, k = [k_nope; k_pe broadcast over heads],
+  scaled scores, additive mask (causal), softmax, weighted sum of v.
+* "DeepSeek-V3.2-Exp - Key-value latent", the MLA-init excerpt: softmax_scale is
+  qk_head_dim^-0.5 with qk_head_dim = qk_nope_head_dim + qk_rope_head_dim.
+* "Value up-projection", "Parameters": 8,388,608 parameters per value up-projection.
+* "DeepSeek V3" (rainlin-net), "Decoupled RoPE": MLA cache = B N (d_c + d_R) s bytes,
+  against 2 B N h_q d_h s for standard MHA.
+
+Readings where the pages are silent (each listed in the design notes):
+* Mask semantics: a scatter of 0 into a -inf row is a set, so a repeated index counts once.
+* Causal prefill: query position s attends keys t <= s.
+* One query token per sequence in decode; the query is the last cached position.
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+
+def _f64(x) -> np.ndarray:
+    """Upcast a numpy array or a CPU torch tensor (any float dtype) to float64."""
+    if hasattr(x, "detach"):  # torch tensor: go through float32 (exact for bf16/fp32)
+        x = x.detach().to("cpu").float().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------------------
+# Weights
+# ----------------------------------------------------------------------------------------
+
+def split_wkv_b(w_kv_b, n_h: int, d_h: int, d_v: int):
+    """Split the fused up-projection into W^UK and W^UV per head.
+
+    "KV Reconstruction", "Official code": wkv_b has shape (n_h (d_h + d_v), d_c), is viewed as
+    (n_h, d_h + d_v, d_c); rows [0, d_h) of each head are W^UK_i and rows [d_h, d_h + d_v) are
+    W^UV_i ("Value up-projection", "Explanation": output features 128-255 of each head's 256).
+
+    Returns (w_uk [n_h, d_h, d_c], w_uv [n_h, d_v, d_c]) as float64.
+    """
+    w = _f64(w_kv_b)
+    d_c = w.shape[-1]
+    assert w.shape == (n_h * (d_h + d_v), d_c), w.shape
+    w = w.reshape(n_h, d_h + d_v, d_c)
+    return w[:, :d_h, :], w[:, d_h:, :]
+
+
+def value_up_params(n_h: int, d_v: int, d_c: int) -> int:
+    """Parameter count of W^UV ("Value up-projection", "Parameters": n_h d_v x d_c)."""
+    return n_h * d_v * d_c
+
+
+def mla_cache_bytes(B: int, N: int, d_c: int, d_r: int, s: int) -> int:
+    """MLA cache size B N (d_c + d_R) s ("DeepSeek V3", "Decoupled RoPE")."""
+    return B * N * (d_c + d_r) * s
+
+
+def mha_cache_bytes(B: int, N: int, h_q: int, d_h: int, s: int) -> int:
+    """Standard MHA cache size 2 B N h_q d_h s, the page's comparison ("Decoupled RoPE")."""
+    return 2 * B * N * h_q * d_h * s
+
+
+# ----------------------------------------------------------------------------------------
+# Softmax and masks
+# ----------------------------------------------------------------------------------------
+
+def softmax(s: np.ndarray, axis: int = -1) -> np.ndarray:
+    """Row softmax, max-subtracted, in float64.  -inf entries get weight 0; every row must
+    hold at least one finite entry."""
+    s = np.asarray(s, dtype=np.float64)
+    m = np.max(s, axis=axis, keepdims=True)
+    assert np.all(np.isfinite(m)), "a softmax row has no finite score"
+    e = np.exp(s - m)
+    return e / np.sum(e, axis=axis, keepdims=True)
+
+
+def _logsumexp(s: np.ndarray, axis: int = -1) -> np.ndarray:
+    m = np.max(s, axis=axis, keepdims=True)
+    return (m + np.log(np.sum(np.exp(s - m), axis=axis, keepdims=True))).squeeze(axis)
+
+
+def index_mask(length: int, topk) -> np.ndarray:
+    """The sparse-attention mask of the V3.2 decode excerpt ("Absorb key weights"): a row of
+    -inf of the cache length with 0 written at every top-k index.  A repeated index writes the
+    same 0 twice, so the selected positions form a set."""
+    mask = np.full((length,), -np.inf, dtype=np.float64)
+    idx = np.asarray(topk, dtype=np.int64).reshape(-1)
+    assert idx.size == 0 or (idx.min() >= 0 and idx.max() < length), "top-k index out of range"
+    mask[idx] = 0.0
+    return mask
+
+
+# ----------------------------------------------------------------------------------------
+# Naive path (the literal equations): the definition everything else is checked against
+# ----------------------------------------------------------------------------------------
+
+def naive_decode(q_nope, q_pe, c_kv, k_r, w_kv_b, scale: float, topk=None, heads=None):
+    """Naive MLA decode for ONE sequence and one query token.
+
+    q_nope [n_h, d_h], q_pe [n_h, d_r], c_kv [L, d_c] and k_r [L, d_r] hold the L cached
+    positions (already cut to the sequence length), w_kv_b [n_h (d_h + d_v), d_c].
+    ``heads`` optionally restricts the evaluation to a subset of heads (heads are independent).
+
+    Steps ("KV Reconstruction", "How it works" and "Naive path"):
+      1. k^C_t = W^UK c_t and v^C_t = W^UV c_t, split into heads       (eqs. 2 and 5)
+      2. k_{t,i} = [k^C_{t,i}; k^R_t]                                  (key assembly)
+      3. q_i = [q^C_i; q^R_i]
+      4. s_{t,i} = scale * q_i . k_{t,i}
+      5. sparse variant: s = -inf outside the top-k set                ("Absorb key weights")
+      6. alpha = softmax over t
+      7. o_i = sum_t alpha_{t,i} v^C_{t,i}
+    Returns (o [n_heads, d_v], alpha [n_heads, L]).
+    """
+    q_nope, q_pe, c_kv, k_r = map(_f64, (q_nope, q_pe, c_kv, k_r))
+    n_h, d_h = q_nope.shape
+    L, d_c = c_kv.shape
+    w = _f64(w_kv_b)
+    d_v = w.shape[0] // n_h - d_h
+    w_uk, w_uv = split_wkv_b(w, n_h, d_h, d_v)
+    hs = np.arange(n_h) if heads is None else np.asarray(heads)
+    # 1. reconstruction: W^UK c_t for every cached t (a plain matmul per head set)
+    k_c = np.einsum("hdc,tc->thd", w_uk[hs], c_kv)           # [L, nh', d_h]
+    v_c = np.einsum("hdc,tc->thd", w_uv[hs], c_kv)           # [L, nh', d_v]
+    # 2. k = [k^C ; k^R] (k^R shared by all heads)
+    k = np.concatenate([k_c, np.broadcast_to(k_r[:, None, :], (L, len(hs), k_r.shape[1]))], axis=-1)
+    # 3. q = [q^C ; q^R]
+    q = np.concatenate([q_nope[hs], q_pe[hs]], axis=-1)       # [nh', d_h + d_r]
+    # 4. scores
+    s = scale * np.einsum("hd,thd->ht", q, k)                # [nh', L]
+    # 5. sparse mask
+    if topk is not None:
+        s = s + index_mask(L, topk)[None, :]
+    # 6. softmax over positions
+    alpha = softmax(s, axis=-1)
+    # 7. weighted sum of the reconstructed values
+    o = np.einsum("ht,thd->hd", alpha, v_c)
+    return o, alpha
+
+
+def naive_prefill(q, c_kv, k_r, w_kv_b, scale: float, n_h: int, d_h: int, d_v: int,
+                  causal: bool = True, rows=None, heads=None):
+    """Naive MLA prefill for ONE sequence ("Value up-projection", MHA-prefill excerpt).
+
+    q [S, n_h, d_h + d_r] (content part first, rotary part last), c_kv [S, d_c], k_r [S, d_r].
+    ``rows`` / ``heads`` optionally restrict which query positions / heads are evaluated; each
+    output row is its own softmax, so this is a subset of the same definition.
+
+    Steps: kv = W_kv_b c (viewed [S, n_h, d_h + d_v]) -> k_nope, v; k = [k_nope; k_pe broadcast];
+    scores = q . k * scale; causal additive mask (t <= s kept); softmax over t; out = sum alpha v.
+    Returns out [len(rows), len(heads), d_v].
+    """
+    q, c_kv, k_r = map(_f64, (q, c_kv, k_r))
+    S = c_kv.shape[0]
+    w = _f64(w_kv_b)
+    rs = np.arange(S) if rows is None else np.asarray(rows)
+    hs = np.arange(n_h) if heads is None else np.asarray(heads)
+    kv = (c_kv @ w.T).reshape(S, n_h, d_h + d_v)[:, hs, :]     # wkv_b(kv), view as heads
+    k_nope, v = kv[..., :d_h], kv[..., d_h:]
+    k = np.concatenate([k_nope, np.broadcast_to(k_r[:, None, :], (S, len(hs), k_r.shape[1]))], axis=-1)
+    qs = q[rs][:, hs, :]                                       # [R, nh', d_h + d_r]
+    scores = np.einsum("rhd,thd->rht", qs, k) * scale          # [R, nh', S]
+    if causal:
+        t = np.arange(S)[None, :]
+        mask = np.where(t <= rs[:, None], 0.0, -np.inf)        # [R, S]
+        scores = scores + mask[:, None, :]
+    alpha = softmax(scores, axis=-1)
+    return np.einsum("rht,thd->rhd", alpha, v)
+
+
+# ----------------------------------------------------------------------------------------
+# Absorbed path, step by step (the three entry points of the decode pipeline)
+# ----------------------------------------------------------------------------------------
+
+def absorb_q(q_nope, w_kv_b, n_h: int, d_h: int, d_v: int) -> np.ndarray:
+    """q~_i = (W^UK_i)^T q^C_i: d_h content features become d_c latent features
+    ("Absorb key weights", first einsum of the decode excerpt).  q_nope [..., n_h, d_h]."""
+    w_uk, _ = split_wkv_b(w_kv_b, n_h, d_h, d_v)
+    return np.einsum("...hd,hdc->...hc", _f64(q_nope), w_uk)
+
+
+def latent_attention(q_tilde, q_pe, c_kv, k_r, scale: float, topk=None):
+    """Attention taken directly over the cached latent for ONE sequence and one query token.
+
+    q_tilde [n_h, d_c], q_pe [n_h, d_r], c_kv [L, d_c], k_r [L, d_r] (cut to the length).
+    s = scale (q~ . c_t + q_pe . k^R_t); optional top-k -inf mask; alpha = softmax over t;
+    ctx = sum_t alpha_t c_t  ("Absorb key weights" decode excerpt; "KV Reconstruction",
+    "Absorb path").  Returns (ctx [n_h, d_c], lse [n_h], alpha [n_h, L]) where lse is the natural
+    log of sum_t exp(s_t) over the kept positions (s already scaled).
+    """
+    q_tilde, q_pe, c_kv, k_r = map(_f64, (q_tilde, q_pe, c_kv, k_r))
+    s = scale * (q_tilde @ c_kv.T + q_pe @ k_r.T)
+    if topk is not None:
+        s = s + index_mask(c_kv.shape[0], topk)[None, :]
+    alpha = softmax(s, axis=-1)
+    return alpha @ c_kv, _logsumexp(s, axis=-1), alpha
+
+
+def out_up(ctx, w_kv_b, n_h: int, d_h: int, d_v: int) -> np.ndarray:
+    """o_i = W^UV_i ctx_i: map the latent context back to d_v value features per head
+    ("Absorb key weights", last einsum of the decode excerpt).  ctx [..., n_h, d_c]."""
+    _, w_uv = split_wkv_b(w_kv_b, n_h, d_h, d_v)
+    return np.einsum("...hc,hdc->...hd", _f64(ctx), w_uv)
+
+
+def absorbed_decode(q_nope, q_pe, c_kv, k_r, w_kv_b, scale: float, d_v: int, topk=None):
+    """The whole absorbed decode for ONE sequence: absorb_q -> latent_attention -> out_up.
+    Returns a dict with q_tilde, ctx, lse, alpha and o (all float64, no intermediate rounding)."""
+    n_h, d_h = np.shape(q_nope)
+    qt = absorb_q(q_nope, w_kv_b, n_h, d_h, d_v)
+    ctx, lse, alpha = latent_attention(qt, q_pe, c_kv, k_r, scale, topk)
+    return {"q_tilde": qt, "ctx": ctx, "lse": lse, "alpha": alpha,
+            "o": out_up(ctx, w_kv_b, n_h, d_h, d_v)}
+
+
+def softmax_scale(d_h: int, d_r: int) -> float:
+    """qk_head_dim^-0.5 with qk_head_dim = d_h + d_r ("Key-value latent", MLA-init excerpt)."""
+    return 1.0 / math.sqrt(d_h + d_r)
