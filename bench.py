@@ -1,0 +1,314 @@
+"""Benchmark of one absorbed MLA decode step: mla_absorb_q -> mla_decode_absorb -> mla_out_up.
+
+Workload: DeepSeek-V3 absorbed decode, B=32 sequences per GPU, 4096 cached positions each,
+128 heads, d_c=512, d_R=64, bf16 storage / fp32 accumulation (synthetic seeded data).
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference]
+
+One JSON line on rank 0.  `value` = decoded tokens per second over all ranks (each rank runs
+its own batch of sequences: batch-sharded replicas, no collective on the data path), timed
+on the device with CUDA events around every step, L2 flushed between steps, max over ranks.
+`--impl reference` times the CPU oracle on the same workload instead (rank 0 only).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from head_latent_attention_absorb_b200.configs import V3_DECODE  # noqa: E402
+from head_latent_attention_absorb_b200.inputs import make_decode_inputs  # noqa: E402
+
+METRIC = "MLA absorbed-decode tokens/s and % of roofline (B=32, N=4096, 128 heads)"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def work_per_step(cfg, lengths):
+    """Algorithmic FLOPs and bytes of each call of one step (bf16 = 2 bytes)."""
+    n_h, d_c, d_r, d_h, d_v, B = cfg.n_h, cfg.d_c, cfg.d_r, cfg.d_h, cfg.d_v, cfg.B
+    tot = int(lengths.sum())
+    w_half = n_h * d_h * d_c * 2
+    return {
+        "absorb_q": {"flops": 2 * B * n_h * d_h * d_c, "bytes": w_half + B * n_h * (d_h + d_c) * 2},
+        "decode": {"flops": 2 * tot * n_h * (d_c + d_r) + 2 * tot * n_h * d_c,
+                   "bytes": tot * (d_c + d_r) * 2 + B * n_h * (d_c + d_r) * 2 + B * n_h * d_c * 2},
+        "out_up": {"flops": 2 * B * n_h * d_c * d_v, "bytes": w_half + B * n_h * (d_c + d_v) * 2},
+    }
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": float(rows[0][2]),
+                "reasons": reasons, "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows)}
+
+
+def cpu_oracle_rate(x, seconds: float, max_seqs: int):
+    """Time the oracle's absorbed decode, one sequence at a time, for about `seconds`."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # pragma: no cover
+        cores = os.cpu_count()
+    cfg = x["cfg"]
+    n, t0 = 0, time.perf_counter()
+    while n < max_seqs:
+        b = n % cfg.B
+        L = int(x["lengths"][b])
+        O.absorbed_decode(x["q_nope"][b], x["q_pe"][b], x["c_kv"][b, :L], x["k_r"][b, :L], x["w_kv_b"],
+                          cfg.scale, cfg.d_v)
+        n += 1
+        if time.perf_counter() - t0 >= seconds:
+            break
+    dt = time.perf_counter() - t0
+    return n / dt, n, dt, cores
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: each step = a bounded sample of the workload."""
+    if rank != 0:
+        return
+    cfg = V3_DECODE
+    x = make_decode_inputs(cfg)
+    # a bounded sample per step: about two minutes for the whole run, at least one sequence
+    _, _, t_one, _ = cpu_oracle_rate(x, 1e9, 1)
+    per_step = max(1, min(cfg.B, int(args.ref_budget_s / ((args.steps + args.warmup) * t_one))))
+    for _ in range(args.warmup):
+        cpu_oracle_rate(x, 1e9, per_step)
+    times, cores = [], 1
+    for _ in range(args.steps):
+        rate, n, dt, cores = cpu_oracle_rate(x, 1e9, per_step)
+        times.append(dt / n)
+    s_per_seq = statistics.mean(times)
+    value = 1.0 / s_per_seq
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_per_seq * cfg.B * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "B": cfg.B, "n_max": cfg.n_max, "n_h": cfg.n_h, "d_c": cfg.d_c,
+                       "d_r": cfg.d_r, "parallelism": "rank 0 only (CPU)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": f"{per_step} of the {cfg.B} sequences per step, absorbed fp64 form"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank, world, local_rank):
+    from head_latent_attention_absorb_b200 import api
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = V3_DECODE
+    x = make_decode_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    dims = cfg.dims
+    B = cfg.B
+    cache = x["cache"].to(dev)
+    c_kv, k_r = cache[..., :cfg.d_c], cache[..., cfg.d_c:]
+    w = x["w_kv_b"].to(dev)
+    q_nope, q_pe, lengths = x["q_nope"].to(dev), x["q_pe"].to(dev), x["lengths"].to(dev)
+    q_tilde = torch.empty((B, cfg.n_h, cfg.d_c), dtype=torch.bfloat16, device=dev)
+    ctx = torch.empty_like(q_tilde)
+    lse = torch.empty((B, cfg.n_h), dtype=torch.float32, device=dev)
+    out = torch.empty((B, cfg.n_h, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((api.mla_decode_workspace_size(dims, torch.bfloat16, B, cfg.n_max),), dtype=torch.uint8,
+                     device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    n_launch = 2 + api.mla_decode_num_launches(dims, torch.bfloat16, B, cfg.n_max)
+
+    def step(qn, qp):
+        api.mla_absorb_q(dims, qn, w, q_tilde, stream=stream)
+        ev[1].record(stream)
+        api.mla_decode_absorb(dims, q_tilde, qp, c_kv, k_r, lengths, cfg.scale, ctx=ctx, lse=lse, workspace=ws,
+                              dev_err=err, stream=stream)
+        ev[2].record(stream)
+        api.mla_out_up(dims, ctx, w, out, stream=stream)
+
+    # ---- device-resident timing ------------------------------------------------------------
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K + args.warmup)]
+    for i in range(args.warmup):
+        ev = evs[i]
+        flush.zero_()
+        ev[0].record(stream); step(q_nope, q_pe); ev[3].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        t_wall = time.perf_counter()
+        for i in range(args.warmup, args.warmup + K):
+            ev = evs[i]
+            flush.zero_()
+            ev[0].record(stream); step(q_nope, q_pe); ev[3].record(stream)
+        torch.cuda.synchronize()
+        t_wall = time.perf_counter() - t_wall
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    per = {"step": [], "absorb_q": [], "decode": [], "out_up": []}
+    for ev in evs[args.warmup:]:
+        per["step"].append(ev[0].elapsed_time(ev[3]))
+        per["absorb_q"].append(ev[0].elapsed_time(ev[1]))
+        per["decode"].append(ev[1].elapsed_time(ev[2]))
+        per["out_up"].append(ev[2].elapsed_time(ev[3]))
+    ms = {k: statistics.mean(v) for k, v in per.items()}
+    assert api.mla_get_device_error(err) == 0, "device error flag raised during the bench"
+
+    # ---- end to end through the public API with host buffers ---------------------------------
+    qn_h = x["q_nope"].pin_memory()
+    qp_h = x["q_pe"].pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    qn_d, qp_d = torch.empty_like(q_nope), torch.empty_like(q_pe)
+    h2d = qn_h.numel() * qn_h.element_size() + qp_h.numel() * qp_h.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+    e2e_ms = []
+    for i in range(args.warmup + K):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        flush.zero_()
+        e0 = torch.cuda.Event(enable_timing=True); e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        qn_d.copy_(qn_h, non_blocking=True)
+        qp_d.copy_(qp_h, non_blocking=True)
+        step(qn_d, qp_d)
+        out_h.copy_(out, non_blocking=True)
+        e1.record(stream)
+        e1.synchronize()
+        if i >= args.warmup:
+            e2e_ms.append(e0.elapsed_time(e1))
+    e2e = statistics.mean(e2e_ms)
+
+    # ---- max over ranks -----------------------------------------------------------------------
+    vals = torch.tensor([ms["step"], ms["decode"], e2e, ms["absorb_q"], ms["out_up"]], dtype=torch.float64,
+                        device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
+    ms_step, ms_dec, ms_e2e, ms_abs, ms_up = vals.tolist()
+    if rank != 0:
+        return
+
+    peaks = load_peaks()
+    work = work_per_step(cfg, x["lengths"])
+    dec = work["decode"]
+    achieved_gbs = dec["bytes"] / (ms_dec * 1e-3) / 1e9
+    achieved_tf = dec["flops"] / (ms_dec * 1e-3) / 1e12
+    clocks = clk.summary()
+    cpu_rate, cpu_n, cpu_dt, cores = cpu_oracle_rate(x, args.cpu_seconds, 10 ** 6)
+    line = {
+        "metric": METRIC, "value": world * B / (ms_step * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": cfg.name, "B_per_gpu": B, "n_max": cfg.n_max, "n_h": cfg.n_h, "d_c": cfg.d_c,
+                   "d_r": cfg.d_r, "d_h": cfg.d_h, "d_v": cfg.d_v, "global_batch": world * B,
+                   "parallelism": f"batch-sharded replicas x{world}", "l2": "flushed (256 MiB write) before each step",
+                   "timing": "CUDA events around each step, mean over steps, max over ranks"},
+        "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mla_decode_absorb",
+                     "peak_source": peaks["source"] + " (hbm_gbs, burst)",
+                     "algorithmic_bytes_per_launch": dec["bytes"], "ms_per_launch": ms_dec,
+                     "tensor_achieved_tflops": achieved_tf, "tensor_peak_tflops": peaks["bf16_tflops"],
+                     "tensor_frac": achieved_tf / peaks["bf16_tflops"]},
+        "per_call_ms": {"absorb_q": ms_abs, "decode": ms_dec, "out_up": ms_up},
+        "cpu_baseline": {"value": cpu_rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{cpu_n} sequences of this workload, fp64 absorbed form, {cpu_dt:.1f} s"},
+        "e2e": {"value": world * B / (ms_e2e * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "note": "queries copied from pinned host memory and outputs read back every step; cache and "
+                        "wkv_b resident"},
+        "gpu_launches": n_launch * K,
+        "clocks": clocks,
+        "wall_s_timed_region": t_wall,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-budget-s", type=float, default=120.0)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,65 @@
+// Shared helpers of the MLA CUDA library: element conversion, warp reductions, the device error
+// flag and the argument blocks handed from the C-ABI layer to the kernel launchers.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "mla_api.h"
+
+namespace mla {
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// First error wins: a later error never overwrites an earlier one.
+__device__ __forceinline__ void raise_error(int32_t* flag, int32_t code) {
+  if (flag != nullptr) atomicCAS(flag, 0, code);
+}
+
+// Validated arguments of one decode call (pointers already checked on the host).
+struct DecodeArgs {
+  int n_h, d_c, d_r, B, n_max, topk;
+  const void* q_tilde; int64_t ldqt;
+  const void* q_pe;    int64_t ldqp;
+  const void* c_kv;    int64_t ckv_b, ckv_r;
+  const void* k_r;     int64_t kr_b, kr_r;
+  const int32_t* lengths;
+  const int32_t* topk_idx;
+  float scale;
+  void* ctx;
+  float* lse;
+  int32_t* err;
+};
+
+struct PrefillArgs {
+  int n_h, d_c, d_r, d_h, d_v, B, S, causal;
+  const void* q;
+  const void* c_kv; int64_t ckv_r;
+  const void* k_r;  int64_t kr_r;
+  const void* w;
+  float scale;
+  void* out;
+  void* kv;  // expanded [B, S, n_h, d_h + d_v] in the input dtype
+};
+
+}  // namespace mla

@@ -1,0 +1,27 @@
+// Kernel launchers behind the C-ABI (internal to libmla_b200.so).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace mla {
+
+// ---- CUDA-core kernels, any dimensions (fp32 element type) -------------------------------
+template <typename T>
+cudaError_t absorb_q_simt_launch(int n_h, int d_c, int d_h, int d_v, int B, const void* q, int64_t ldq,
+                                 const void* w, void* qt, cudaStream_t st);
+template <typename T>
+cudaError_t out_up_simt_launch(int n_h, int d_c, int d_h, int d_v, int B, const void* ctx, const void* w,
+                               void* out, cudaStream_t st);
+template <typename T>
+cudaError_t decode_simt_launch(const DecodeArgs& a, void* ws, cudaStream_t st);
+template <typename T>
+cudaError_t prefill_simt_launch(const PrefillArgs& a, cudaStream_t st);
+
+int decode_simt_splits(int B, int n_keys_cap);
+size_t decode_simt_workspace(int n_h, int d_c, int B, int n_keys_cap);
+
+}  // namespace mla

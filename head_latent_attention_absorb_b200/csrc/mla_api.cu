@@ -1,0 +1,239 @@
+// C-ABI entry points of libmla_b200.so: host-side validation, then dispatch to the kernels.
+// Every check that can be made on the host is made here, before anything is launched.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "mla_api.h"
+
+namespace {
+
+thread_local char g_msg[512] = "";
+
+mla_status fail(mla_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+mla_status cuda_status(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return MLA_OK;
+  return fail(MLA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool is_deepseek(const mla_dims& d) {
+  return d.n_h == 128 && d.d_c == 512 && d.d_r == 64 && d.d_h == 128 && d.d_v == 128;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+mla_status check_dims(const mla_dims& d, mla_dtype dt) {
+  if (d.n_h <= 0 || d.d_c <= 0 || d.d_r <= 0 || d.d_h <= 0 || d.d_v <= 0)
+    return fail(MLA_ERR_INVALID_ARG, "dimensions must be positive (n_h=%d d_c=%d d_r=%d d_h=%d d_v=%d)",
+                d.n_h, d.d_c, d.d_r, d.d_h, d.d_v);
+  if (dt == MLA_BF16) {
+    if (!is_deepseek(d))
+      return fail(MLA_ERR_UNSUPPORTED, "bf16 kernels need n_h=128 d_c=512 d_r=64 d_h=d_v=128");
+    return MLA_OK;
+  }
+  if (dt == MLA_F32) {
+    if (d.n_h > 1024 || d.d_c > 1024 || d.d_r > 128 || d.d_h > 256 || d.d_v > 256)
+      return fail(MLA_ERR_UNSUPPORTED, "fp32 kernels accept n_h, d_c <= 1024, d_r <= 128, d_h, d_v <= 256");
+    return MLA_OK;
+  }
+  return fail(MLA_ERR_INVALID_ARG, "unknown dtype %d", (int)dt);
+}
+
+// bf16 operands feed 16-byte vector loads and TMA: pointers 16-byte aligned, strides 8-element multiples
+mla_status check_bf16_ptr(mla_dtype dt, const void* p, const char* name) {
+  if (dt == MLA_BF16 && !aligned16(p)) return fail(MLA_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  return MLA_OK;
+}
+mla_status check_bf16_stride(mla_dtype dt, int64_t s, const char* name) {
+  if (dt == MLA_BF16 && (s % 8) != 0) return fail(MLA_ERR_INVALID_ARG, "%s must be a multiple of 8 elements", name);
+  return MLA_OK;
+}
+
+#define MLA_TRY(x)                   \
+  do {                               \
+    mla_status _s = (x);             \
+    if (_s != MLA_OK) return _s;     \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int32_t mla_abi_version(void) { return MLA_ABI_VERSION; }
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: invalid argument";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: no kernel for these dimensions / dtype";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA: CUDA runtime error";
+    case MLA_ERR_INDEX: return "MLA_ERR_INDEX: top-k index outside [0, length)";
+    case MLA_ERR_TIMEOUT: return "MLA_ERR_TIMEOUT: bounded wait in a kernel ran out";
+    case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace missing or too small";
+    case MLA_ERR_LENGTH: return "MLA_ERR_LENGTH: sequence length outside [1, n_max]";
+  }
+  return "unknown mla_status";
+}
+
+const char* mla_last_error_message(void) { return g_msg; }
+
+mla_status mla_absorb_q(mla_dims dims, mla_dtype dtype, int32_t B, const void* q_nope, int64_t ldq,
+                        const void* w_kv_b, void* q_tilde, void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0) return fail(MLA_ERR_INVALID_ARG, "B must be positive");
+  if (!q_nope || !w_kv_b || !q_tilde) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (ldq < dims.d_h) return fail(MLA_ERR_INVALID_ARG, "ldq < d_h");
+  MLA_TRY(check_bf16_ptr(dtype, q_nope, "q_nope"));
+  MLA_TRY(check_bf16_ptr(dtype, w_kv_b, "w_kv_b"));
+  MLA_TRY(check_bf16_ptr(dtype, q_tilde, "q_tilde"));
+  MLA_TRY(check_bf16_stride(dtype, ldq, "ldq"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == MLA_BF16)
+    e = mla::absorb_q_simt_launch<__nv_bfloat16>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, q_nope, ldq, w_kv_b,
+                                                 q_tilde, st);
+  else
+    e = mla::absorb_q_simt_launch<float>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, q_nope, ldq, w_kv_b, q_tilde, st);
+  return cuda_status(e, "mla_absorb_q launch");
+}
+
+size_t mla_decode_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
+  if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
+  const int cap = topk > 0 ? topk : n_max;
+  return mla::decode_simt_workspace(dims.n_h, dims.d_c, B, cap);
+}
+
+int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
+  if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
+  const int cap = topk > 0 ? topk : n_max;
+  return mla::decode_simt_splits(B, cap) > 1 ? 2 : 1;
+}
+
+mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B, const void* q_tilde, int64_t ldqt,
+                             const void* q_pe, int64_t ldqp, const void* c_kv, int64_t ckv_bstride,
+                             int64_t ckv_rstride, const void* k_r, int64_t kr_bstride, int64_t kr_rstride,
+                             int32_t n_max, const int32_t* lengths, const int32_t* topk_idx, int32_t topk,
+                             float scale, void* ctx_out, float* lse_out, void* workspace, size_t ws_bytes,
+                             int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0 || n_max <= 0) return fail(MLA_ERR_INVALID_ARG, "B and n_max must be positive");
+  if (!q_tilde || !q_pe || !c_kv || !k_r || !lengths || !ctx_out)
+    return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (topk_idx && (topk < 1 || topk > n_max)) return fail(MLA_ERR_INVALID_ARG, "topk must lie in [1, n_max]");
+  if (ldqt < dims.d_c || ldqp < dims.d_r) return fail(MLA_ERR_INVALID_ARG, "query row stride too small");
+  if (ckv_rstride < dims.d_c || kr_rstride < dims.d_r || ckv_bstride < 0 || kr_bstride < 0)
+    return fail(MLA_ERR_INVALID_ARG, "cache stride too small");
+  if (!(scale > 0.f) || scale != scale) return fail(MLA_ERR_INVALID_ARG, "scale must be positive");
+  MLA_TRY(check_bf16_ptr(dtype, q_tilde, "q_tilde"));
+  MLA_TRY(check_bf16_ptr(dtype, q_pe, "q_pe"));
+  MLA_TRY(check_bf16_ptr(dtype, c_kv, "c_kv"));
+  MLA_TRY(check_bf16_ptr(dtype, k_r, "k_r"));
+  MLA_TRY(check_bf16_ptr(dtype, ctx_out, "ctx_out"));
+  MLA_TRY(check_bf16_stride(dtype, ldqt, "ldqt"));
+  MLA_TRY(check_bf16_stride(dtype, ldqp, "ldqp"));
+  MLA_TRY(check_bf16_stride(dtype, ckv_bstride, "ckv_bstride"));
+  MLA_TRY(check_bf16_stride(dtype, ckv_rstride, "ckv_rstride"));
+  MLA_TRY(check_bf16_stride(dtype, kr_bstride, "kr_bstride"));
+  MLA_TRY(check_bf16_stride(dtype, kr_rstride, "kr_rstride"));
+  const size_t need = mla_decode_workspace_size(dims, dtype, B, n_max, topk_idx ? topk : 0);
+  if (!workspace || ws_bytes < need)
+    return fail(MLA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace ? ws_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+
+  mla::DecodeArgs a;
+  a.n_h = dims.n_h; a.d_c = dims.d_c; a.d_r = dims.d_r; a.B = B; a.n_max = n_max;
+  a.topk = topk_idx ? topk : 0;
+  a.q_tilde = q_tilde; a.ldqt = ldqt; a.q_pe = q_pe; a.ldqp = ldqp;
+  a.c_kv = c_kv; a.ckv_b = ckv_bstride; a.ckv_r = ckv_rstride;
+  a.k_r = k_r; a.kr_b = kr_bstride; a.kr_r = kr_rstride;
+  a.lengths = lengths; a.topk_idx = topk_idx; a.scale = scale;
+  a.ctx = ctx_out; a.lse = lse_out; a.err = dev_err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == MLA_BF16 ? mla::decode_simt_launch<__nv_bfloat16>(a, workspace, st)
+                                    : mla::decode_simt_launch<float>(a, workspace, st);
+  return cuda_status(e, "mla_decode_absorb launch");
+}
+
+mla_status mla_out_up(mla_dims dims, mla_dtype dtype, int32_t B, const void* ctx, const void* w_kv_b, void* out,
+                      void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0) return fail(MLA_ERR_INVALID_ARG, "B must be positive");
+  if (!ctx || !w_kv_b || !out) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  MLA_TRY(check_bf16_ptr(dtype, ctx, "ctx"));
+  MLA_TRY(check_bf16_ptr(dtype, w_kv_b, "w_kv_b"));
+  MLA_TRY(check_bf16_ptr(dtype, out, "out"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (dtype == MLA_BF16)
+    e = mla::out_up_simt_launch<__nv_bfloat16>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, ctx, w_kv_b, out, st);
+  else
+    e = mla::out_up_simt_launch<float>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, ctx, w_kv_b, out, st);
+  return cuda_status(e, "mla_out_up launch");
+}
+
+size_t mla_prefill_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S) {
+  if (check_dims(dims, dtype) != MLA_OK || B <= 0 || S <= 0) return 0;
+  const size_t es = dtype == MLA_BF16 ? 2 : 4;
+  return (size_t)B * S * dims.n_h * (dims.d_h + dims.d_v) * es;
+}
+
+mla_status mla_prefill_naive(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S, const void* q, const void* c_kv,
+                             int64_t ckv_rstride, const void* k_r, int64_t kr_rstride, const void* w_kv_b,
+                             float scale, int32_t causal, void* out, void* workspace, size_t ws_bytes,
+                             void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0 || S <= 0) return fail(MLA_ERR_INVALID_ARG, "B and S must be positive");
+  if (!q || !c_kv || !k_r || !w_kv_b || !out) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (ckv_rstride < dims.d_c || kr_rstride < dims.d_r) return fail(MLA_ERR_INVALID_ARG, "row stride too small");
+  if (!(scale > 0.f)) return fail(MLA_ERR_INVALID_ARG, "scale must be positive");
+  MLA_TRY(check_bf16_ptr(dtype, q, "q"));
+  MLA_TRY(check_bf16_ptr(dtype, c_kv, "c_kv"));
+  MLA_TRY(check_bf16_ptr(dtype, k_r, "k_r"));
+  MLA_TRY(check_bf16_ptr(dtype, w_kv_b, "w_kv_b"));
+  MLA_TRY(check_bf16_ptr(dtype, out, "out"));
+  MLA_TRY(check_bf16_stride(dtype, ckv_rstride, "ckv_rstride"));
+  MLA_TRY(check_bf16_stride(dtype, kr_rstride, "kr_rstride"));
+  const size_t need = mla_prefill_workspace_size(dims, dtype, B, S);
+  if (!workspace || ws_bytes < need)
+    return fail(MLA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace ? ws_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  mla::PrefillArgs a;
+  a.n_h = dims.n_h; a.d_c = dims.d_c; a.d_r = dims.d_r; a.d_h = dims.d_h; a.d_v = dims.d_v;
+  a.B = B; a.S = S; a.causal = causal ? 1 : 0;
+  a.q = q; a.c_kv = c_kv; a.ckv_r = ckv_rstride; a.k_r = k_r; a.kr_r = kr_rstride; a.w = w_kv_b;
+  a.scale = scale; a.out = out; a.kv = workspace;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = dtype == MLA_BF16 ? mla::prefill_simt_launch<__nv_bfloat16>(a, st)
+                                    : mla::prefill_simt_launch<float>(a, st);
+  return cuda_status(e, "mla_prefill_naive launch");
+}
+
+mla_status mla_clear_device_error(int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  if (!dev_err) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  return cuda_status(cudaMemsetAsync(dev_err, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream)),
+                     "mla_clear_device_error");
+}
+
+mla_status mla_get_device_error(const int32_t* dev_err, int32_t* host_out) {
+  g_msg[0] = 0;
+  if (!dev_err || !host_out) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  MLA_TRY(cuda_status(cudaDeviceSynchronize(), "mla_get_device_error sync"));
+  return cuda_status(cudaMemcpy(host_out, dev_err, sizeof(int32_t), cudaMemcpyDeviceToHost),
+                     "mla_get_device_error copy");
+}
+
+}  // extern "C"

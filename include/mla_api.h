@@ -1,0 +1,178 @@
+/*
+ * mla_api.h - C ABI of libmla_b200.so: multi-head latent attention (MLA) for NVIDIA B200 (sm_100a).
+ *
+ * The four operations are the steps of DeepSeek-V3 / V3.2 MLA as the pages state them:
+ *   mla_absorb_q       q~_i = (W^UK_i)^T q^C_i                       ("Absorb key weights", first einsum)
+ *   mla_decode_absorb  softmax over cached positions of
+ *                      scale (q~ . c^KV_t + q^R . k^R_t), weighted sum of c^KV_t
+ *                                                                    ("Absorb key weights", decode excerpt)
+ *   mla_out_up         o_i = W^UV_i ctx_i                            ("Absorb key weights", last einsum)
+ *   mla_prefill_naive  wkv_b expansion, k = [k_nope; k^R], causal attention
+ *                                                                    ("Value up-projection", prefill excerpt;
+ *                                                                     "KV Reconstruction", "Naive path")
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Every data pointer is a DEVICE pointer owned by the caller; the library allocates nothing,
+ *   keeps no pointer after a call returns and never synchronises the stream (except the two
+ *   calls documented as blocking).  `stream` is a cudaStream_t (NULL = legacy default stream).
+ * - Element type: MLA_BF16 (bf16 storage, fp32 accumulation) or MLA_F32 (fp32 throughout,
+ *   no TF32).  Integer tensors are int32.  Strides are in ELEMENTS.
+ * - W_kv_b is the fused up-projection ("KV Reconstruction", "How it works" and "Official code"):
+ *   row-major [n_h * (d_h + d_v), d_c]; rows [i(d_h+d_v), i(d_h+d_v)+d_h) of head i are W^UK_i,
+ *   the next d_v rows are W^UV_i ("Value up-projection", "Explanation").
+ * - MLA_BF16 runs the tcgen05 tensor-core kernels, specialised for the DeepSeek-V3 dimensions
+ *   n_h=128, d_c=512, d_r=64, d_h=d_v=128; other bf16 dimensions return MLA_ERR_UNSUPPORTED.
+ *   bf16 pointers must be 16-byte aligned and row strides multiples of 8 elements.
+ *   MLA_F32 accepts any dimensions with n_h <= 1024, d_c <= 1024, d_r <= 128, d_h, d_v <= 256.
+ * - Host-checkable errors (NULL pointer, bad size, alignment, workspace too small) return at
+ *   once and launch nothing.  Data-dependent errors found by a kernel (a length outside
+ *   [1, n_max], a top-k index outside [0, length)) are written to the optional device flag
+ *   `dev_err` (first error wins) and the offending row is skipped; kernels never trap.
+ */
+#ifndef MLA_API_H
+#define MLA_API_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MLA_ABI_VERSION 1
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive size, misaligned pointer or stride  */
+  MLA_ERR_UNSUPPORTED = 2,  /* dimensions / dtype combination without a kernel               */
+  MLA_ERR_CUDA = 3,         /* a CUDA runtime call failed (see mla_last_error_message)       */
+  MLA_ERR_INDEX = 4,        /* device flag: a top-k index outside [0, length)                */
+  MLA_ERR_TIMEOUT = 5,      /* device flag: a bounded wait inside a kernel ran out           */
+  MLA_ERR_WORKSPACE = 6,    /* workspace NULL or smaller than the matching *_workspace_size  */
+  MLA_ERR_LENGTH = 7        /* device flag: a sequence length outside [1, n_max]             */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+/* Head count and widths ("Key-value latent", MLA-init excerpt): n_h heads, latent d_c
+ * (kv_lora_rank), rotary width d_r (qk_rope_head_dim), content key width d_h
+ * (qk_nope_head_dim), value width d_v (v_head_dim).  DeepSeek-V3: {128, 512, 64, 128, 128}. */
+typedef struct {
+  int32_t n_h, d_c, d_r, d_h, d_v;
+} mla_dims;
+
+/* ABI version of the loaded library (MLA_ABI_VERSION when the header matches). */
+int32_t mla_abi_version(void);
+
+/* Static text for a status code; never NULL. */
+const char* mla_status_string(mla_status s);
+
+/* Details of the last host-side error raised on the calling thread ("" if none). */
+const char* mla_last_error_message(void);
+
+/*
+ * mla_absorb_q - fold W^UK into each head's content query ("Absorb key weights": 128 content
+ * features become 512 latent features; "KV Reconstruction", "Absorb path").
+ *   q_nope   [B, n_h, d_h], element (b,h,d) at q_nope[(b*n_h + h)*ldq + d]   (ldq >= d_h)
+ *   w_kv_b   [n_h*(d_h+d_v), d_c] row-major (only the W^UK rows are read)
+ *   q_tilde  [B, n_h, d_c] contiguous output, q_tilde[b,h,c] = sum_d q_nope[b,h,d] W^UK_h[d,c]
+ * Asynchronous on `stream`.
+ */
+mla_status mla_absorb_q(mla_dims dims, mla_dtype dtype, int32_t B,
+                        const void* q_nope, int64_t ldq, const void* w_kv_b,
+                        void* q_tilde, void* stream);
+
+/*
+ * mla_decode_workspace_size - bytes of scratch mla_decode_absorb needs for this shape on the
+ * current device (split-KV partial results and the split plan).  An upper bound for any
+ * lengths <= n_max; 0 never means "no workspace needed" for B > 0.
+ */
+size_t mla_decode_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk);
+
+/*
+ * mla_decode_num_launches - how many kernels one mla_decode_absorb call with these sizes
+ * launches on the current device (the split-KV plan decides whether a combine pass runs).
+ * 0 for arguments mla_decode_absorb would reject.
+ */
+int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk);
+
+/*
+ * mla_decode_absorb - attention of one query token per sequence over its latent cache
+ * ("Absorb key weights", decode excerpt; "KV Reconstruction", "Absorb path").
+ *   For sequence b with length L_b = lengths[b] and every head h:
+ *     s_t   = scale * (q_tilde[b,h,:] . c_kv[b,t,:] + q_pe[b,h,:] . k_r[b,t,:])
+ *     kept positions: t in [0, L_b), or, when topk_idx != NULL, the set {topk_idx[b, j]} (the
+ *     -inf scatter mask of the V3.2 sparse variant; indices must be distinct, in [0, L_b))
+ *     ctx[b,h,:] = sum_t softmax(s)_t c_kv[b,t,:],   lse[b,h] = log sum_t exp(s_t)
+ *   q_tilde  [B, n_h, d_c], element (b,h,c) at q_tilde[(b*n_h + h)*ldqt + c]
+ *   q_pe     [B, n_h, d_r], element (b,h,r) at q_pe[(b*n_h + h)*ldqp + r]
+ *   c_kv     row t of sequence b at c_kv + b*ckv_bstride + t*ckv_rstride (d_c elements)
+ *   k_r      row t of sequence b at k_r + b*kr_bstride + t*kr_rstride (d_r elements)
+ *            (a packed [B, n_max, d_c + d_r] cache is c_kv = base, k_r = base + d_c, both
+ *             row strides d_c + d_r)
+ *   n_max    cache capacity per sequence; lengths (device, int32 [B]) must lie in [1, n_max]
+ *   topk_idx NULL (dense) or device int32 [B, topk]; 1 <= topk <= n_max
+ *   scale    softmax scale, (d_h + d_r)^-0.5 for DeepSeek ("Key-value latent", MLA-init)
+ *   ctx_out  [B, n_h, d_c] contiguous, dtype as the inputs
+ *   lse_out  NULL or float [B, n_h] (natural log)
+ *   workspace/ws_bytes  device scratch of at least mla_decode_workspace_size() bytes; its
+ *            contents need no initialisation and are garbage afterwards
+ *   dev_err  NULL or a device int32 flag; MLA_ERR_LENGTH / MLA_ERR_INDEX are stored there
+ * Asynchronous on `stream`.
+ */
+mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
+                             const void* q_tilde, int64_t ldqt, const void* q_pe, int64_t ldqp,
+                             const void* c_kv, int64_t ckv_bstride, int64_t ckv_rstride,
+                             const void* k_r, int64_t kr_bstride, int64_t kr_rstride,
+                             int32_t n_max, const int32_t* lengths,
+                             const int32_t* topk_idx, int32_t topk,
+                             float scale, void* ctx_out, float* lse_out,
+                             void* workspace, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/*
+ * mla_out_up - map the latent context back up through W^UV ("Absorb key weights", last einsum;
+ * "KV Reconstruction", "Absorb path": W^UV applied after the weighted sum).
+ *   ctx  [B, n_h, d_c] contiguous;  out [B, n_h, d_v] contiguous,
+ *   out[b,h,d] = sum_c ctx[b,h,c] W^UV_h[d,c]   (only the W^UV rows of w_kv_b are read)
+ * Asynchronous on `stream`.
+ */
+mla_status mla_out_up(mla_dims dims, mla_dtype dtype, int32_t B,
+                      const void* ctx, const void* w_kv_b, void* out, void* stream);
+
+/*
+ * mla_prefill_workspace_size - bytes of scratch mla_prefill_naive needs: the expanded
+ * [B, S, n_h, d_h + d_v] keys/values in the input dtype.
+ */
+size_t mla_prefill_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S);
+
+/*
+ * mla_prefill_naive - the naive path over a whole sequence ("Value up-projection", prefill
+ * excerpt; "KV Reconstruction", "Naive path"):
+ *   kv[b,s,h,:] = W_kv_b c_kv[b,s,:]  viewed as [d_h | d_v] -> k_nope, v
+ *   k[b,t,h,:]  = [k_nope[b,t,h,:]; k_r[b,t,:]]        (k_r shared by all heads)
+ *   out[b,s,h,:] = sum_t softmax_t(scale q[b,s,h,:] . k[b,t,h,:] + mask) v[b,t,h,:]
+ *   mask: causal != 0 keeps t <= s (the additive causal mask); causal == 0 keeps every t.
+ *   q     [B, S, n_h, d_h + d_r] contiguous (content part first, rotary part last)
+ *   c_kv  row s of sequence b at c_kv + (b*S + s)*ckv_rstride;  k_r likewise with kr_rstride
+ *   out   [B, S, n_h, d_v] contiguous
+ *   workspace/ws_bytes  at least mla_prefill_workspace_size() bytes (holds the expansion)
+ * Asynchronous on `stream`.
+ */
+mla_status mla_prefill_naive(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S,
+                             const void* q, const void* c_kv, int64_t ckv_rstride,
+                             const void* k_r, int64_t kr_rstride, const void* w_kv_b,
+                             float scale, int32_t causal, void* out,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* Zero the device flag (asynchronous on `stream`). */
+mla_status mla_clear_device_error(int32_t* dev_err, void* stream);
+
+/* BLOCKING: wait for all work on the current device, then copy the device flag to *host_out. */
+mla_status mla_get_device_error(const int32_t* dev_err, int32_t* host_out);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_API_H */

@@ -1,0 +1,96 @@
+"""The C-ABI library builds, loads and exports every entry point include/mla_api.h declares;
+host-side validation answers without touching a GPU (no call here reaches a kernel launch)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from head_latent_attention_absorb_b200 import _capi
+from head_latent_attention_absorb_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+DS = _capi.MLADims(128, 512, 64, 128, 128)
+FAKE = 0x10000  # an aligned non-NULL address; every call below fails validation before using it
+
+
+@pytest.fixture(scope="module")
+def L():
+    build(quiet=True)
+    return _capi.lib()
+
+
+def declared_functions():
+    names = []
+    for h in HEADERS:
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(mla_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 11, names
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in include/ but not exported"
+        assert n in _capi.SIGNATURES, f"{n} has no ctypes signature"
+
+
+def test_abi_and_status_strings(L):
+    assert L.mla_abi_version() == _capi.ABI_VERSION
+    for code, name in _capi.STATUS.items():
+        assert L.mla_status_string(code).decode().startswith(name)
+    assert L.mla_status_string(99) == b"unknown mla_status"
+
+
+def test_workspace_sizes(L):
+    assert L.mla_prefill_workspace_size(DS, _capi.MLA_BF16, 2, 2048) == 2 * 2048 * 128 * 256 * 2
+    assert L.mla_prefill_workspace_size(_capi.MLADims(4, 64, 16, 32, 32), _capi.MLA_F32, 1, 9) == 9 * 4 * 64 * 4
+    assert L.mla_decode_workspace_size(DS, _capi.MLA_BF16, 32, 4096, 0) > 0
+    assert L.mla_decode_workspace_size(DS, _capi.MLA_BF16, 0, 4096, 0) == 0
+    assert L.mla_decode_workspace_size(_capi.MLADims(4, 64, 16, 32, 32), _capi.MLA_BF16, 1, 64, 0) == 0
+
+
+def test_host_validation_codes(L):
+    bf, f32 = _capi.MLA_BF16, _capi.MLA_F32
+    tiny = _capi.MLADims(4, 64, 16, 32, 32)
+    # bf16 outside the DeepSeek dimensions has no kernel
+    assert L.mla_absorb_q(tiny, bf, 1, FAKE, 32, FAKE, FAKE, None) == 2
+    # NULL pointers, bad sizes, misalignment
+    assert L.mla_absorb_q(DS, bf, 1, None, 128, FAKE, FAKE, None) == 1
+    assert L.mla_absorb_q(DS, bf, 0, FAKE, 128, FAKE, FAKE, None) == 1
+    assert L.mla_absorb_q(DS, bf, 1, FAKE + 2, 128, FAKE, FAKE, None) == 1
+    assert L.mla_absorb_q(DS, bf, 1, FAKE, 100, FAKE, FAKE, None) == 1
+    assert b"ldq" in L.mla_last_error_message() or b"multiple" in L.mla_last_error_message()
+    assert L.mla_out_up(DS, bf, 1, FAKE, None, FAKE, None) == 1
+    assert L.mla_absorb_q(_capi.MLADims(0, 64, 16, 32, 32), f32, 1, FAKE, 32, FAKE, FAKE, None) == 1
+    assert L.mla_absorb_q(tiny, 7, 1, FAKE, 32, FAKE, FAKE, None) == 1
+
+    def dec(**kw):
+        a = dict(dims=DS, dt=bf, B=2, qt=FAKE, ldqt=512, qp=FAKE, ldqp=64, ckv=FAKE, cb=4096 * 576, cr=576,
+                 kr=FAKE, kb=4096 * 576, krr=576, n_max=4096, lengths=FAKE, topk=None, k=0, scale=0.07,
+                 ctx=FAKE, lse=None, ws=FAKE, wsb=1 << 40, err=None)
+        a.update(kw)
+        return L.mla_decode_absorb(*a.values(), None)
+
+    assert dec(ws=None) == 6
+    assert dec(wsb=16) == 6
+    assert dec(lengths=None) == 1
+    assert dec(cr=500) == 1                 # row stride below d_c
+    assert dec(cr=577) == 1                 # not a multiple of 8 elements
+    assert dec(topk=FAKE, k=0) == 1         # top-k with an empty set
+    assert dec(topk=FAKE, k=4097) == 1      # top-k larger than the cache
+    assert dec(scale=0.0) == 1
+    assert dec(scale=float("nan")) == 1
+    assert dec(ldqt=256) == 1
+    assert dec(B=0) == 1
+    # prefill
+    assert L.mla_prefill_naive(DS, bf, 1, 16, FAKE, FAKE, 576, FAKE, 576, FAKE, 0.07, 1, FAKE, None, 0, None) == 6
+    assert L.mla_prefill_naive(DS, bf, 1, 0, FAKE, FAKE, 576, FAKE, 576, FAKE, 0.07, 1, FAKE, FAKE, 1 << 30, None) == 1
+    assert L.mla_clear_device_error(None, None) == 1
+    out = ctypes.c_int32(0)
+    assert L.mla_get_device_error(None, ctypes.byref(out)) == 1
