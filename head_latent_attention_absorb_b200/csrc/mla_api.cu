@@ -110,12 +110,18 @@ mla_status mla_absorb_q(mla_dims dims, mla_dtype dtype, int32_t B, const void* q
 size_t mla_decode_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
   if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
   const int cap = topk > 0 ? topk : n_max;
-  return mla::decode_simt_workspace(dims.n_h, dims.d_c, B, cap);
+  size_t ws = mla::decode_simt_workspace(dims.n_h, dims.d_c, B, cap);
+  if (dtype == MLA_BF16 && topk == 0) {
+    const size_t tc = mla::decode_tc_workspace(B);
+    ws = tc > ws ? tc : ws;
+  }
+  return ws;
 }
 
 int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
   if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
   const int cap = topk > 0 ? topk : n_max;
+  if (dtype == MLA_BF16 && topk == 0) return 2;  // tensor-core decode + combine
   return mla::decode_simt_splits(B, cap) > 1 ? 2 : 1;
 }
 
@@ -160,8 +166,13 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B, const vo
   a.lengths = lengths; a.topk_idx = topk_idx; a.scale = scale;
   a.ctx = ctx_out; a.lse = lse_out; a.err = dev_err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = dtype == MLA_BF16 ? mla::decode_simt_launch<__nv_bfloat16>(a, workspace, st)
-                                    : mla::decode_simt_launch<float>(a, workspace, st);
+  cudaError_t e;
+  if (dtype == MLA_BF16 && !topk_idx)
+    e = mla::decode_tc_launch(a, workspace, st);
+  else if (dtype == MLA_BF16)
+    e = mla::decode_simt_launch<__nv_bfloat16>(a, workspace, st);
+  else
+    e = mla::decode_simt_launch<float>(a, workspace, st);
   return cuda_status(e, "mla_decode_absorb launch");
 }
 
