@@ -109,13 +109,10 @@ mla_status mla_absorb_q(mla_dims dims, mla_dtype dtype, int32_t B, const void* q
 
 size_t mla_decode_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
   if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
+  // bf16 dense decode runs the tensor-core kernel only; every other case the CUDA-core kernels
+  if (dtype == MLA_BF16 && topk == 0) return mla::decode_tc_workspace(B);
   const int cap = topk > 0 ? topk : n_max;
-  size_t ws = mla::decode_simt_workspace(dims.n_h, dims.d_c, B, cap);
-  if (dtype == MLA_BF16 && topk == 0) {
-    const size_t tc = mla::decode_tc_workspace(B);
-    ws = tc > ws ? tc : ws;
-  }
-  return ws;
+  return mla::decode_simt_workspace(dims.n_h, dims.d_c, B, cap);
 }
 
 int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
