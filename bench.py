@@ -29,6 +29,7 @@ sys.path.insert(0, ROOT)
 
 from head_latent_attention_absorb_b200.configs import V3_DECODE  # noqa: E402
 from head_latent_attention_absorb_b200.inputs import make_decode_inputs  # noqa: E402
+from head_latent_attention_absorb_b200.shard import max_over_ranks, shard_range  # noqa: E402
 
 METRIC = "MLA absorbed-decode tokens/s and % of roofline (B=32, N=4096, 128 heads)"
 UNIT = "tokens/s"
@@ -158,7 +159,10 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cfg = V3_DECODE
-    x = make_decode_inputs(cfg, seed=cfg.seed + 1000 * rank)
+    # this rank's share of the global batch (world x B sequences); each share has its own cache
+    first_seq, n_seq = shard_range(world * cfg.B, world, rank)
+    assert n_seq == cfg.B
+    x = make_decode_inputs(cfg, seed=cfg.seed + first_seq)
     dims = cfg.dims
     B = cfg.B
     cache = x["cache"].to(dev)
@@ -239,11 +243,8 @@ def run_ours(args, rank, world, local_rank):
     e2e = statistics.mean(e2e_ms)
 
     # ---- max over ranks -----------------------------------------------------------------------
-    vals = torch.tensor([ms["step"], ms["decode"], e2e, ms["absorb_q"], ms["out_up"]], dtype=torch.float64,
-                        device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(vals, op=torch.distributed.ReduceOp.MAX)
-    ms_step, ms_dec, ms_e2e, ms_abs, ms_up = vals.tolist()
+    ms_step, ms_dec, ms_e2e, ms_abs, ms_up = max_over_ranks(
+        [ms["step"], ms["decode"], e2e, ms["absorb_q"], ms["out_up"]], device=dev)
     if rank != 0:
         return
 
