@@ -111,6 +111,29 @@ def mla_decode_absorb(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_kv: tor
     return ctx
 
 
+def mla_decode_absorb_static(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_kv: torch.Tensor,
+                             k_r: torch.Tensor, lengths: torch.Tensor, scale: float,
+                             ctx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                             dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """bf16 dense decode with the library's built-in scratch (for callers that cannot allocate a
+    workspace).  `ctx` (and `lse`) are allocated here only when not given."""
+    d = _dims(dims)
+    B, n_max = c_kv.shape[0], c_kv.shape[1]
+    ldqt, ldqp = _headrows(q_tilde, "q_tilde"), _headrows(q_pe, "q_pe")
+    _rows(c_kv, "c_kv")
+    _rows(k_r, "k_r")
+    if lengths.dtype != torch.int32:
+        raise TypeError("lengths must be int32")
+    if ctx is None:
+        ctx = torch.empty((B, d.n_h, d.d_c), dtype=q_tilde.dtype, device=q_tilde.device)
+    check(lib().mla_decode_absorb_static(
+        d, _dt(q_tilde), B, _ptr(q_tilde), ldqt, _ptr(q_pe), ldqp,
+        _ptr(c_kv), c_kv.stride(0), c_kv.stride(1), _ptr(k_r), k_r.stride(0), k_r.stride(1),
+        n_max, _ptr(lengths), float(scale), _ptr(ctx), _ptr(lse), _ptr(dev_err), _stream(stream)),
+        "mla_decode_absorb_static")
+    return ctx
+
+
 def mla_out_up(dims, ctx: torch.Tensor, w_kv_b: torch.Tensor, out: Optional[torch.Tensor] = None,
                stream=None) -> torch.Tensor:
     """o[b,h,:] = W^UV_h ctx[b,h,:].  ctx [B, n_h, d_c] contiguous."""

@@ -35,6 +35,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
@@ -770,6 +772,47 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   combine_kernel<<<dim3(a.B, kNH / 8), 256, 0, st>>>(p);
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------------------
+// Built-in scratch of mla_decode_absorb_static
+// ------------------------------------------------------------------------------------------
+// Some callers cannot allocate device memory when they run a decode: a plugin or engine host
+// whose enqueue callback may not call cudaMalloc (it would synchronise or break the host's memory
+// budget), code issuing work while a stream is being captured into a CUDA graph, or a caller that
+// only holds pointers handed to it by someone else.  For them the split-KV scratch lives in this
+// file-scope array, which every GPU that loads the library holds until the process exits.
+// Sized for 74 clusters (one CTA pair per two SMs of a 148-SM B200): 74 x 2 partial slots of
+// 128 heads x 512 fp32 features, their (m, l) pairs and the per-cluster plan, about 37.1 MiB.
+namespace {
+constexpr size_t kStaticMaxClusters = 74;
+constexpr size_t kStaticScratchBytes = 2 * kStaticMaxClusters * (2 * 128 * 256 * sizeof(float)) +
+                                       2 * kStaticMaxClusters * 128 * sizeof(float2) +
+                                       kStaticMaxClusters * sizeof(int32_t) + 1024;
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+}  // namespace
+
+size_t decode_static_scratch_bytes() { return kStaticScratchBytes; }
+
+// Device address of the array on the current device.  Host code may not use the array's name as a
+// device pointer (it is a host-side stand-in), so the address is looked up once per device, with
+// that device current, and cached.
+cudaError_t decode_static_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {nullptr};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return cudaSuccess;
 }
 
 }  // namespace mla

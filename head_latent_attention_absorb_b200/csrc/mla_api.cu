@@ -173,6 +173,29 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B, const vo
   return cuda_status(e, "mla_decode_absorb launch");
 }
 
+mla_status mla_decode_absorb_static(mla_dims dims, mla_dtype dtype, int32_t B, const void* q_tilde, int64_t ldqt,
+                                    const void* q_pe, int64_t ldqp, const void* c_kv, int64_t ckv_bstride,
+                                    int64_t ckv_rstride, const void* k_r, int64_t kr_bstride, int64_t kr_rstride,
+                                    int32_t n_max, const int32_t* lengths, float scale, void* ctx_out,
+                                    float* lse_out, int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  if (dtype != MLA_BF16)
+    return fail(MLA_ERR_UNSUPPORTED, "mla_decode_absorb_static covers the bf16 dense decode only");
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0 || n_max <= 0) return fail(MLA_ERR_INVALID_ARG, "B and n_max must be positive");
+  const size_t need = mla_decode_workspace_size(dims, dtype, B, n_max, 0);
+  const size_t have = mla::decode_static_scratch_bytes();
+  if (need > have)
+    return fail(MLA_ERR_WORKSPACE,
+                "mla_decode_absorb_static: this device needs %zu bytes of split-KV scratch, the built-in "
+                "scratch holds %zu (it is sized for up to 148 SMs)", need, have);
+  void* scratch = nullptr;
+  MLA_TRY(cuda_status(mla::decode_static_scratch(&scratch), "mla_decode_absorb_static scratch set-up"));
+  return mla_decode_absorb(dims, dtype, B, q_tilde, ldqt, q_pe, ldqp, c_kv, ckv_bstride, ckv_rstride, k_r,
+                           kr_bstride, kr_rstride, n_max, lengths, nullptr, 0, scale, ctx_out, lse_out, scratch,
+                           have, dev_err, stream);
+}
+
 mla_status mla_out_up(mla_dims dims, mla_dtype dtype, int32_t B, const void* ctx, const void* w_kv_b, void* out,
                       void* stream) {
   g_msg[0] = 0;

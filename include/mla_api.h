@@ -131,6 +131,31 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
                              void* workspace, size_t ws_bytes, int32_t* dev_err, void* stream);
 
 /*
+ * mla_decode_absorb_static - mla_decode_absorb for the bf16 dense decode (no top-k) WITHOUT a
+ * caller-supplied workspace.  The pages have no counterpart: this is a deployment convenience.
+ *   For callers that cannot allocate device memory around a decode call: a plugin / engine host
+ *   whose enqueue path may not call cudaMalloc, code issuing work while a stream is being captured
+ *   into a CUDA graph, or a caller that only holds pointers handed to it.  The split-KV scratch is
+ *   a file-scope device array of 38,950,184 bytes (about 37.1 MiB: 74 clusters x 2 partial slots),
+ *   held by every GPU that loads the library until the process exits.
+ *   Arguments and results are those of mla_decode_absorb with topk_idx = NULL and without
+ *   workspace / ws_bytes.  dtype must be MLA_BF16 (else MLA_ERR_UNSUPPORTED); a device that would
+ *   need more scratch than the array holds (more than 148 SMs) gets MLA_ERR_WORKSPACE.
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
+ *   that device current) and caches it; make that first call before any stream capture begins.
+ *   Every call shares the one array and it keeps the last call's contents; nothing in it needs to
+ *   start at zero (each byte a call reads was written earlier in the same call), but calls whose
+ *   work overlaps on the GPU (different streams, or different host threads) race on it: serialise
+ *   them.  No allocation of any kind happens inside this call.  Asynchronous on `stream`.
+ */
+mla_status mla_decode_absorb_static(mla_dims dims, mla_dtype dtype, int32_t B,
+                                    const void* q_tilde, int64_t ldqt, const void* q_pe, int64_t ldqp,
+                                    const void* c_kv, int64_t ckv_bstride, int64_t ckv_rstride,
+                                    const void* k_r, int64_t kr_bstride, int64_t kr_rstride,
+                                    int32_t n_max, const int32_t* lengths, float scale,
+                                    void* ctx_out, float* lse_out, int32_t* dev_err, void* stream);
+
+/*
  * mla_out_up - map the latent context back up through W^UV ("Absorb key weights", last einsum;
  * "KV Reconstruction", "Absorb path": W^UV applied after the weighted sum).
  *   ctx  [B, n_h, d_c] contiguous;  out [B, n_h, d_v] contiguous,
