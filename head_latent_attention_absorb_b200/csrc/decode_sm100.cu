@@ -40,6 +40,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "sm100_ptx.cuh"
+#include "tma_host.h"
 
 namespace mla {
 namespace decode_tc {
@@ -631,64 +632,65 @@ __global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ Pa
     return;
   }
   if (c_lo == c_hi) return;  // one cluster held the whole sequence and wrote ctx itself
-  const long long total = s_info[3], nc = p.n_clusters;
-  for (int i = threadIdx.x; i < 8 * (kDC / 4); i += blockDim.x) {
-    const int hh = h0 + i / (kDC / 4), d = (i % (kDC / 4)) * 4;
-    float M = -INFINITY;
-    for (int c = c_lo; c <= c_hi; ++c) {
-      if (range_lo(c, total, nc) == range_lo(c + 1, total, nc)) continue;  // empty range: no partial
-      const int slot = 2 * c + (p.ws_plan[c] == b ? 0 : 1);
-      M = fmaxf(M, p.ws_ml[(int64_t)slot * kNH + hh].x);
+  // ---- the partial slots of this sequence, resolved once (clusters with an empty range hold none)
+  constexpr int kMaxSlots = 256;
+  __shared__ int s_slot[kMaxSlots];
+  __shared__ int s_nslot;
+  __shared__ float s_w[8][kMaxSlots];  // per head: e^{m_s - M} / L, the weight of partial s
+  if (threadIdx.x == 0) {
+    const long long total = s_info[3], nc = p.n_clusters;
+    int ns = 0;
+    long long lo = range_lo(c_lo, total, nc);
+    for (int c = c_lo; c <= c_hi && ns < kMaxSlots; ++c) {
+      const long long hi = range_lo(c + 1, total, nc);
+      if (hi > lo) s_slot[ns++] = 2 * c + (p.ws_plan[c] == b ? 0 : 1);
+      lo = hi;
     }
+    s_nslot = ns;
+  }
+  __syncthreads();
+  const int ns = s_nslot;
+  {  // one warp per head: running-max merge of (m_s, l_s)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hh = h0 + warp;
+    float M = -INFINITY;
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.ws_ml[(int64_t)s_slot[s] * kNH + hh].x);
+    M = warp_max(M);
     float L = 0.f;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = c_lo; c <= c_hi; ++c) {
-      if (range_lo(c, total, nc) == range_lo(c + 1, total, nc)) continue;
-      const int slot = 2 * c + (p.ws_plan[c] == b ? 0 : 1);
-      const float2 ml = p.ws_ml[(int64_t)slot * kNH + hh];
+    for (int s = lane; s < ns; s += 32) {
+      const float2 ml = p.ws_ml[(int64_t)s_slot[s] * kNH + hh];
       const float w = ex2(ml.x - M);
+      s_w[warp][s] = w;
       L += w * ml.y;
+    }
+    L = warp_sum(L);
+    const float inv = 1.f / L;
+    for (int s = lane; s < ns; s += 32) s_w[warp][s] *= inv;
+    if (lane == 0 && p.lse) p.lse[(int64_t)b * kNH + hh] = (M + log2f(L)) * 0.69314718055994531f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 8 * (kDC / 4); i += blockDim.x) {
+    const int hl = i / (kDC / 4), hh = h0 + hl, d = (i % (kDC / 4)) * 4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 0; s < ns; ++s) {
+      const float w = s_w[hl][s];
       const float4 o = *reinterpret_cast<const float4*>(
-          p.ws_o + (((int64_t)slot * 2 + (d >> 8)) * kNH + hh) * 256 + (d & 255));
+          p.ws_o + (((int64_t)s_slot[s] * 2 + (d >> 8)) * kNH + hh) * 256 + (d & 255));
       acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
     }
-    const float inv = 1.f / L;
     __nv_bfloat16* out = p.ctx + ((int64_t)b * kNH + hh) * kDC + d;
-    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(acc.x * inv, acc.y * inv), pack_bf16x2(acc.z * inv, acc.w * inv));
-    if (d == 0 && p.lse) p.lse[(int64_t)b * kNH + hh] = (M + log2f(L)) * 0.69314718055994531f;
+    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
   }
 }
 
 // ------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* f = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(f);
-  }
-  return fn;
-}
-
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
                  uint64_t s2_bytes, uint32_t box0, uint32_t box1, CUtensorMapSwizzle sw) {
-  EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
-  const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {s1_bytes, s2_bytes};
-  const cuuint32_t box[3] = {box0, box1, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const uint64_t dims[3] = {d0, d1, d2};
+  const uint64_t strides[2] = {s1_bytes, s2_bytes};
+  const uint32_t box[3] = {box0, box1, 1};
+  return make_tensor_map_bf16(m, base, 3, dims, strides, box, sw);
 }
 
 size_t smem_bytes() { return (size_t)kStages * kStageBytes + 2 * kXBytes + sizeof(Smem) + 1024; }

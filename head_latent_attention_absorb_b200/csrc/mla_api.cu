@@ -100,8 +100,7 @@ mla_status mla_absorb_q(mla_dims dims, mla_dtype dtype, int32_t B, const void* q
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (dtype == MLA_BF16)
-    e = mla::absorb_q_simt_launch<__nv_bfloat16>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, q_nope, ldq, w_kv_b,
-                                                 q_tilde, st);
+    e = mla::absorb_q_tc_launch(B, q_nope, ldq, w_kv_b, q_tilde, st);
   else
     e = mla::absorb_q_simt_launch<float>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, q_nope, ldq, w_kv_b, q_tilde, st);
   return cuda_status(e, "mla_absorb_q launch");
@@ -208,7 +207,7 @@ mla_status mla_out_up(mla_dims dims, mla_dtype dtype, int32_t B, const void* ctx
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (dtype == MLA_BF16)
-    e = mla::out_up_simt_launch<__nv_bfloat16>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, ctx, w_kv_b, out, st);
+    e = mla::out_up_tc_launch(B, ctx, w_kv_b, out, st);
   else
     e = mla::out_up_simt_launch<float>(dims.n_h, dims.d_c, dims.d_h, dims.d_v, B, ctx, w_kv_b, out, st);
   return cuda_status(e, "mla_out_up launch");
