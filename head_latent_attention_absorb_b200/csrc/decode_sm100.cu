@@ -49,15 +49,17 @@ using namespace sm100;
 
 constexpr int kNH = 128, kDC = 512, kDR = 64;
 constexpr int kTile = 64;                       // keys per tile
-constexpr int kStages = 5;
+constexpr int kStages = 4;
 constexpr int kSlabBytes = kTile * 128;         // 64 rows x 64 latent features (bf16)
 constexpr int kLatBytes = 4 * kSlabBytes;       // 256 latent features
 constexpr int kRopeBytes = kTile * 64;          // 64 rows x 32 rotary features
 constexpr int kStageBytes = kLatBytes + kRopeBytes;
 constexpr int kXBytes = kNH * kTile * 2;        // one partial-score exchange buffer (fp16)
-constexpr int kSoftmaxWarps = 8;
-constexpr int kPvWarp = 2 + kSoftmaxWarps;      // the warp that issues the P*V MMAs
-constexpr int kThreads = 32 * (kPvWarp + 1);
+constexpr int kSoftmaxWarps = 8;                // two per TMEM lane quadrant
+constexpr int kPvWarp = 2;                      // the warp that issues the P*V MMAs
+constexpr int kAWarp0 = 3;                      // 4 exchange warps, one per TMEM lane quadrant
+constexpr int kBWarp0 = 7;                      // 8 softmax warps
+constexpr int kThreads = 32 * (kBWarp0 + kSoftmaxWarps);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352;  // Q: 128 + 16 columns
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
@@ -85,6 +87,7 @@ struct Smem {
   uint64_t full[kStages], empty[kStages];
   uint64_t q_full, s_full, s_empty, p_full, pv_done, drain;
   uint64_t x_full[2], x_free[2];   // exchange buffers (double-buffered by tile parity)
+  uint64_t own_ready[2], stg_free[2];  // this CTA's fp16 partial staged / read by the softmax warps
   uint64_t red_bar[2][4], sum_bar; // row-max rendezvous of the two warps of a lane quadrant / final sum
   float red[2][2][kNH];            // [tile parity][key half][head] partial row max
   float lsum[2][kNH];              // [key half][head] partial softmax sum
@@ -191,8 +194,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  float* xbuf = reinterpret_cast<float*>(smem + kStages * kStageBytes);  // [2][128][64]
-  Smem& sm = *reinterpret_cast<Smem*>(smem + kStages * kStageBytes + 2 * kXBytes);
+  uint8_t* xbuf = smem + kStages * kStageBytes;  // 2 receive + 2 staging exchange buffers
+  Smem& sm = *reinterpret_cast<Smem*>(smem + kStages * kStageBytes + 4 * kXBytes);
   volatile int* abort_flag = &sm.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -207,13 +210,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // softmax-side arrivals are one per softmax warp, after a __syncwarp
     mbar_init(smem_u32(&sm.q_full), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.s_full), 1);
-    mbar_init(smem_u32(&sm.s_empty), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.s_empty), 4);  // the four exchange warps
     mbar_init(smem_u32(&sm.p_full), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.pv_done), 1);
     mbar_init(smem_u32(&sm.drain), 2);  // one commit from each MMA-issuing thread
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.x_full[i]), 1);  // 1 local arrive.expect_tx + the peer's st.async bytes
       mbar_init(smem_u32(&sm.x_free[i]), 1);  // 1 remote arrive from the peer
+      mbar_init(smem_u32(&sm.own_ready[i]), 4);
+      mbar_init(smem_u32(&sm.stg_free[i]), kSoftmaxWarps);
       for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&sm.red_bar[i][q]), 2);
     }
     mbar_init(smem_u32(&sm.sum_bar), kSoftmaxWarps);
@@ -326,11 +331,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       __syncwarp();
     };
     // O += P(t) V(t) over this CTA's 256 latent features
-    // P(t) in TMEM also means every softmax warp has read exchange buffer t % 2: tell the peer
-    const uint32_t x_free_peer0 = mapa(smem_u32(&sm.x_free[0]), peer);
     auto issue_pv = [&](uint32_t t, bool first_of_seg) {
       if (!wait_or_fail(smem_u32(&sm.p_full), t & 1u, false)) return;
-      if (lane == 0) mbar_arrive_remote_relaxed(x_free_peer0 + 8 * (t & 1u));
       tc_fence_after();
       const uint32_t st = t % kStages;
       if (lane == 0) {
@@ -359,25 +361,87 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) mma_commit(smem_u32(&sm.drain));
     __syncwarp();
     mbar_wait(smem_u32(&sm.drain), 0, abort_flag, kWaitLimitNs);
+  } else if (warp >= kAWarp0 && warp < kAWarp0 + 4) {
+    // ------------------------------------------------------------------ exchange warps (one per quadrant)
+    // Phase A of every tile: read this CTA's partial S(t) (fp32, 288 features) from TMEM, round it
+    // to fp16 into the staging buffer (the softmax warps read it from there) and bulk-copy the same
+    // 4 KB block to the peer.  Both CTAs then add the same two fp16 halves, so their scores agree
+    // bit for bit (relative rounding 2^-11 per half-score).
+    const int quad = warp & 3;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + kColS;
+    const bool a_leader = (warp == kAWarp0 && lane == 0);
+    const uint32_t xb = smem_u32(xbuf), xb_peer = mapa(xb, peer), stg = xb + 2 * kXBytes;
+    const uint32_t blk = quad * 4096;                          // [quad][key half][32 rows][32 keys]
+    const uint32_t swz = (lane >> 1) & 3;
+    const uint32_t x_full_l0 = smem_u32(&sm.x_full[0]), x_full_r0 = mapa(x_full_l0, peer);
+    bool ok = true;
+    auto wait_or_fail = [&](uint32_t bar, uint32_t par, bool cl_scope) {
+      if (!ok) return false;
+      const bool mine = mbar_wait(bar, par, abort_flag, kWaitLimitNs, cl_scope);
+      if (!__all_sync(0xffffffffu, mine)) {
+        if (lane == 0) fail_timeout(sm, p.err);
+        ok = false;
+      }
+      return ok;
+    };
+    const uint32_t ntiles = sm.hi > sm.lo ? (uint32_t)(sm.hi - sm.lo) : 0u;
+    for (uint32_t t = 0; t < ntiles && ok; ++t) {
+      const uint32_t xi = t & 1u, use = t >> 1;
+      if (!wait_or_fail(smem_u32(&sm.s_full), t & 1u, false)) break;
+      tc_fence_after();
+      uint32_t h16[32];
+      {
+        uint32_t r[32];
+        tmem_ld32(tS, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) h16[k] = pack_f16x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+        tmem_ld32(tS + 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) h16[16 + k] = pack_f16x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty));
+      // staging xi is free once the peer consumed tile t - 2 (so its copy is done) and this CTA's
+      // softmax warps have read it
+      if (!wait_or_fail(smem_u32(&sm.x_free[xi]), (use & 1u) ^ 1u, true)) break;
+      if (!wait_or_fail(smem_u32(&sm.stg_free[xi]), (use & 1u) ^ 1u, false)) break;
+      // The softmax warps release staging xi only after they have waited for receive buffer xi of
+      // tile t - 2, so that phase of x_full[xi] is complete and this tile's expected byte count
+      // opens the next one (never two arrivals in one phase).
+      if (a_leader) mbar_arrive_expect_tx(x_full_l0 + 8 * xi, kXBytes);
+      const uint32_t row = stg + xi * kXBytes + blk + lane * 64;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          st_shared_v4_b32(row + hf * 2048 + ((j ^ swz) << 4), h16[16 * hf + 4 * j], h16[16 * hf + 4 * j + 1],
+                           h16[16 * hf + 4 * j + 2], h16[16 * hf + 4 * j + 3]);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        bulk_copy_to_peer(xb_peer + xi * kXBytes + blk, stg + xi * kXBytes + blk, 4096, x_full_r0 + 8 * xi);
+        mbar_arrive(smem_u32(&sm.own_ready[xi]));
+      }
+    }
   } else {
-    // ------------------------------------------------------------------ softmax warps (2..9)
-    // Scores are exchanged as fp16 partials; each CTA rounds its own partial the same way, so
-    // both hold the identical sum fp16(S_0) + fp16(S_1) (relative rounding 2^-11 per partial).
-    const int sw = warp - 2;
+    // ------------------------------------------------------------------ softmax warps (kBWarp0..)
+    const int sw = warp - kBWarp0;
     const int half = sw >> 2;                        // which 32 keys of each tile
     const int quad = warp & 3;                       // TMEM lane quadrant of this warp
     const int h = quad * 32 + lane;                  // head == TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tO = tmem + lane_off + kColO + 128 * half;   // this half's O columns
-    const uint32_t tS = tmem + lane_off + kColS + 32 * half;
     const uint32_t tP = tmem + lane_off + kColP + 16 * half;
     const uint32_t tQ = tmem + lane_off + kColQ;
-    const bool leader = (sw == 0 && lane == 0);
-    const uint32_t xb = smem_u32(xbuf), xb_peer = mapa(xb, peer);
-    const uint32_t row_off = h * (kTile * 2);  // one 128-byte fp16 row per head
-    // barrier addresses of exchange buffer i are base + 8 i (adjacent array elements)
+    const uint32_t xb = smem_u32(xbuf), stg = xb + 2 * kXBytes;
+    const uint32_t row_off = quad * 4096 + half * 2048 + lane * 64;
+    const uint32_t swz = (lane >> 1) & 3;
     const uint32_t x_full_l0 = smem_u32(&sm.x_full[0]);
-    const uint32_t x_full_r0 = mapa(x_full_l0, peer);
+    const uint32_t x_free_peer0 = mapa(smem_u32(&sm.x_free[0]), peer);
     auto warp_arrive = [&](uint32_t bar) {
       __syncwarp();
       if (lane == 0) mbar_arrive(bar);
@@ -385,7 +449,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     SegIter seg(sm, p);
     int b, begin, end, len;
     bool whole;
-    uint32_t ta = 0, tb = 0;   // global tile counters of phases A and B
+    uint32_t tb = 0;           // global tile counter
     uint32_t nseg = 0;
     bool ok = true;
     bool first_seg = true;     // the first segment of the range uses partial slot 2c, the last 2c + 1
@@ -397,30 +461,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         ok = false;
       }
       return ok;
-    };
-    // Phase A(t): read this CTA's partial S(t), round it to fp16 (the value both CTAs then use)
-    // and ship it to the peer's exchange buffer t % 2.
-    auto phase_a = [&](uint32_t (&ha)[16]) {
-      const uint32_t xi = ta & 1u, use = ta >> 1;
-      if (leader) mbar_arrive_expect_tx(x_full_l0 + 8 * xi, kXBytes);  // the peer's partial of this tile
-      if (!wait_or_fail(smem_u32(&sm.s_full), ta & 1u, false)) return;
-      tc_fence_after();
-      uint32_t r[32];
-      tmem_ld32(tS, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int k = 0; k < 16; ++k) ha[k] = pack_f16x2(__uint_as_float(r[2 * k]), __uint_as_float(r[2 * k + 1]));
-      tc_fence_before();
-      warp_arrive(smem_u32(&sm.s_empty));
-      if (!wait_or_fail(smem_u32(&sm.x_free[xi]), (use & 1u) ^ 1u, true)) return;
-      const uint32_t dst = xb_peer + xi * kXBytes + row_off;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int c = 4 * half + j;  // 16-byte chunk of the 128-byte row, swizzled by head
-        st_async_v4_b32(dst + ((c ^ (h & 7)) << 4), x_full_r0 + 8 * xi, ha[4 * j], ha[4 * j + 1], ha[4 * j + 2],
-                        ha[4 * j + 3]);
-      }
-      ++ta;
     };
     while (ok && seg.next(b, begin, end, len, whole)) {
       // ---- this sequence's query half into TMEM (A operand of the score MMA)
@@ -452,27 +492,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         warp_arrive(smem_u32(&sm.q_full));
       }
       float m_run = -INFINITY, l_run = 0.f;
-      uint32_t ha[16], hn[16];
-      phase_a(ha);
       for (int i = begin; i < end && ok; ++i) {
-        if (i + 1 < end) phase_a(hn);
-        if (!ok) break;
-        // ---- phase B(t): full scores, online softmax (base 2), P into TMEM
+        // ---- full scores of this tile: own fp16 partial (staging) + the peer's (receive buffer)
         const bool first = (i == begin);
         const uint32_t xi = tb & 1u, use = tb >> 1;
+        if (!wait_or_fail(smem_u32(&sm.own_ready[xi]), use & 1u, false)) break;
         if (!wait_or_fail(x_full_l0 + 8 * xi, use & 1u, true)) break;
-        const uint32_t src = xb + xi * kXBytes + row_off;
         float sa[32];
+        {
+          uint4 mine[4], theirs[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int c = 4 * half + j;
-          const uint4 v = ld_shared_v4_b32(src + ((c ^ (h & 7)) << 4));
-          const uint32_t pv[4] = {v.x, v.y, v.z, v.w};
+          for (int j = 0; j < 4; ++j) {
+            mine[j] = ld_shared_v4_b32(stg + xi * kXBytes + row_off + ((j ^ swz) << 4));
+            theirs[j] = ld_shared_v4_b32(xb + xi * kXBytes + row_off + ((j ^ swz) << 4));
+          }
+          warp_arrive(smem_u32(&sm.stg_free[xi]));
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 mine = unpack_f16x2(ha[4 * j + q]), theirs = unpack_f16x2(pv[q]);
-            sa[8 * j + 2 * q] = mine.x + theirs.x;
-            sa[8 * j + 2 * q + 1] = mine.y + theirs.y;
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t a4[4] = {mine[j].x, mine[j].y, mine[j].z, mine[j].w};
+            const uint32_t b4[4] = {theirs[j].x, theirs[j].y, theirs[j].z, theirs[j].w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const float2 s2 = unpack_f16x2(hadd2_u32(a4[q], b4[q]));
+              sa[8 * j + 2 * q] = s2.x;
+              sa[8 * j + 2 * q + 1] = s2.y;
+            }
           }
         }
         const int valid = len - i * kTile - 32 * half;  // keys of this half inside the sequence
@@ -487,6 +531,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int q = 0; q < 4; ++q) mx[q] = fmaxf(mx[q], fmaxf(fmaxf(sa[q + 16], sa[q + 20]), fmaxf(sa[q + 24], sa[q + 28])));
         const float lmax = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        if (sw == 0 && lane == 0) {
+          // all eight softmax warps have read receive buffer xi: the peer may refill it
+          if (mbar_wait(smem_u32(&sm.stg_free[xi]), use & 1u, abort_flag, kWaitLimitNs))
+            mbar_arrive_remote_relaxed(x_free_peer0 + 8 * xi);
+        }
         // rendezvous with the warp holding the other key half of the same heads
         sm.red[xi][half][h] = lmax;
         warp_arrive(smem_u32(&sm.red_bar[xi][quad]));
@@ -531,8 +580,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_before();
         warp_arrive(smem_u32(&sm.p_full));
         ++tb;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) ha[k] = hn[k];
       }
       if (!ok) break;
       // ---- epilogue: O (this CTA's 256 latent features) -> ctx, or a partial for the combine
@@ -693,7 +740,7 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
   return make_tensor_map_bf16(m, base, 3, dims, strides, box, sw);
 }
 
-size_t smem_bytes() { return (size_t)kStages * kStageBytes + 2 * kXBytes + sizeof(Smem) + 1024; }
+size_t smem_bytes() { return (size_t)kStages * kStageBytes + 4 * kXBytes + sizeof(Smem) + 1024; }
 
 // Upper bound of clusters: one CTA pair per two SMs (sizes the workspace).
 int max_clusters() {
