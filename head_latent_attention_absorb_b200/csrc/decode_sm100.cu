@@ -2,32 +2,32 @@
 // sequence directly over the latent cache ("Absorb key weights", decode excerpt:
 // scores = scale (q~ . c^KV_t + q^R . k^R_t), softmax over positions, ctx = sum alpha c^KV_t).
 //
-// Design (one CTA pair = one thread-block cluster of 2 per work range, 1 CTA per SM):
+// Design (one CTA pair = one thread-block cluster of 2, 1 CTA per SM, one wave):
 // * The 128 heads of one sequence are the M = 128 rows of every MMA.
 // * TMEM (512 columns) cannot hold the fp32 context of 128 heads x 512 latent features plus a
 //   score tile, so the pair splits the latent axis: CTA r owns latent features
 //   [256 r, 256 r + 256) and rotary features [32 r, 32 r + 32).  Each CTA loads only its half of
 //   every cached row (no byte is loaded twice), computes the PARTIAL score tile over its 288
-//   features, and the two partials are exchanged through distributed shared memory (st.async,
-//   completion counted on the receiver's mbarrier), so both CTAs hold identical full scores and
-//   run the identical online softmax.
+//   features, and the two partials are exchanged through distributed shared memory as fp16 (bulk
+//   copies completing on the receiver's mbarrier); both CTAs add the same two fp16 halves, so
+//   their scores agree bit for bit and they run the identical online softmax.
 // * Per 64-key tile: TMA brings the CTA's half rows (4 x 128-byte-swizzled slabs + a 64-byte-
 //   swizzled rotary slab) into a 4-stage ring; S = Q K^T runs with Q held in TMEM (A operand)
 //   and K in shared memory; P (bf16) is written to TMEM and O += P V reads V from the SAME
 //   shared-memory tile (K-major for the scores, MN-major for the values).
-// * Softmax: 8 warps, two per TMEM lane quadrant; the two warps of a quadrant split each tile's
-//   64 keys (32 each) and agree on the row maximum through shared memory.  The per-tile work is
-//   software-pipelined: phase A(t) reads S(t) from TMEM and ships the partial to the peer,
-//   phase B(t) adds the peer's partial and does the softmax; the order A(t+1), B(t) keeps one
-//   exchange in flight while the previous tile is normalised, and lets the score MMA of tile
-//   t+1 run while the softmax of tile t-1 is still busy.
+// * Warp roles: warp 0 = TMA producer; warp 1 = TMEM allocator + score-MMA issuer; warp 2 =
+//   P.V-MMA issuer; warps 3..6 = exchange (read S from TMEM, round to fp16, stage, bulk-copy to
+//   the peer); warps 7..14 = softmax (two per TMEM lane quadrant, 32 keys each, agreeing on the
+//   row maximum through shared memory), O rescale and epilogue.
 // * Online softmax in base 2 with the scale folded in; the running maximum is only raised (and
 //   O rescaled in TMEM) when it grows by more than 8, so rescales are rare.
-// * Split-KV: the sequence axis of all sequences is cut into equal contiguous tile ranges, one
-//   per cluster (balanced for ragged lengths); a range that covers a whole sequence writes ctx
-//   directly, the others write fp32 partials (O, m, l) and a combine kernel merges them.
-// * Warp roles: warp 0 = TMA producer, warp 1 = TMEM allocator + MMA issuer, warps 2..9 =
-//   softmax, exchange, rescale and epilogue.
+// * Work split: when every non-empty sequence can get its own clusters, each sequence is cut into
+//   chunks of at most `chunk` tiles and cluster i takes chunk i (one sequence per cluster, so the
+//   query is loaded once, by TMA, and no pipeline restart happens mid-kernel); otherwise the
+//   concatenated tiles of all sequences are cut into equal contiguous ranges.  A cluster that
+//   covers a whole sequence writes ctx directly; the others write fp32 partials (O, m, l) and the
+//   last cluster to finish a sequence (an arrival counter per sequence and latent half) merges
+//   them, so no second kernel is launched.
 // * Every wait is a bounded mbarrier wait (global timer); on expiry the kernel records
 //   MLA_ERR_TIMEOUT, drains and returns.
 #include <cuda.h>
@@ -35,6 +35,8 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+#include <chrono>
 #include <mutex>
 
 #include "common.cuh"
@@ -55,6 +57,13 @@ constexpr int kLatBytes = 4 * kSlabBytes;       // 256 latent features
 constexpr int kRopeBytes = kTile * 64;          // 64 rows x 32 rotary features
 constexpr int kStageBytes = kLatBytes + kRopeBytes;
 constexpr int kXBytes = kNH * kTile * 2;        // one partial-score exchange buffer (fp16)
+constexpr int kQLatBytes = kNH * 256 * 2;       // this CTA's latent half of the query (128 heads)
+constexpr int kQRopeBytes = kNH * 32 * 2;       // this CTA's rotary half of the query
+static_assert(kQLatBytes == 4 * kXBytes, "the first query is staged in the four exchange buffers");
+constexpr int kXOff = kStages * kStageBytes;    // shared-memory layout: stages | exchange | q rope | Smem
+constexpr int kQRopeOff = kXOff + 4 * kXBytes;
+constexpr int kSmemOff = kQRopeOff + kQRopeBytes;
+constexpr int kMaxClusters = 160;               // partial-slot list capacity (2 slots per cluster)
 constexpr int kSoftmaxWarps = 8;                // two per TMEM lane quadrant
 constexpr int kPvWarp = 2;                      // the warp that issues the P*V MMAs
 constexpr int kAWarp0 = 3;                      // 4 exchange warps, one per TMEM lane quadrant
@@ -68,6 +77,8 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 struct Params {
   CUtensorMap tm_ckv;  // 3-D (d_c, n_max, B), box (64, 64, 1), 128-byte swizzle
   CUtensorMap tm_kr;   // 3-D (d_r, n_max, B), box (32, 64, 1), 64-byte swizzle
+  CUtensorMap tm_q;    // 2-D (d_c, B * 128) rows of q~, box (64, 128), 128-byte swizzle
+  CUtensorMap tm_qp;   // 2-D (d_r, B * 128) rows of q^R, box (32, 128), 64-byte swizzle
   const __nv_bfloat16* q_tilde;
   int64_t ldqt;
   const __nv_bfloat16* q_pe;
@@ -77,27 +88,48 @@ struct Params {
   float scale_log2;
   __nv_bfloat16* ctx;
   float* lse;
-  float* ws_o;     // [2 n_clusters slots][2 halves][128][256] fp32, unnormalised
-  float2* ws_ml;   // [2 n_clusters slots][128] (running max in log2 units, sum)
-  int32_t* ws_plan;  // [n_clusters] first sequence of each cluster's range
+  float* ws_o;     // [2 n_clusters slots][2 halves][256 features][128 heads] fp32, unnormalised
+                   // (feature-major, so a warp's 32 heads of one feature are 128 contiguous bytes)
+  float2* ws_ml;   // [2 n_clusters slots][2 halves][128] (running max in log2 units, sum)
+  unsigned long long* ws_ctr;  // [B][2 halves] arrival counters: (epoch << 8) | arrivals
+  unsigned long long epoch;    // unique per launch, never 0, < 2^56
   int32_t* err;
 };
 
 struct Smem {
   uint64_t full[kStages], empty[kStages];
-  uint64_t q_full, s_full, s_empty, p_full, pv_done, drain;
+  uint64_t q_tma, q_full, s_full, s_empty, p_full, pv_done, drain;
   uint64_t x_full[2], x_free[2];   // exchange buffers (double-buffered by tile parity)
   uint64_t own_ready[2], stg_free[2];  // this CTA's fp16 partial staged / read by the softmax warps
   uint64_t red_bar[2][4], sum_bar; // row-max rendezvous of the two warps of a lane quadrant / final sum
+  uint64_t pub_bar, last_bar;      // partial published by all softmax warps / merge decision made
   float red[2][2][kNH];            // [tile parity][key half][head] partial row max
   float lsum[2][kNH];              // [key half][head] partial softmax sum
+  int16_t slots[kMaxClusters];     // partial slots of the sequence being merged
   uint32_t tmem_base;
   int abort;
-  int lo, hi, b0, t_b0;
+  int lo, hi, b0, t_b0;  // tile range [lo, hi) in the global tile order, its first sequence and
+                         // that sequence's first global tile
+  int chunk;             // > 0: chunked plan, every cluster holds <= chunk tiles of one sequence
+  int item0, kb;         // chunked plan: first chunk of this cluster's sequence, its chunk count
+  long long total;       // tiles of all sequences
+  int bad;               // some length outside [1, n_max]
+  int nslots, is_last;
 };
 
 __device__ __forceinline__ int clamp_len(int len, int n_max) { return len < 0 ? 0 : (len > n_max ? n_max : len); }
 __device__ __forceinline__ int tiles_of(int len) { return (len + kTile - 1) / kTile; }
+
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ int warp_max_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -108,25 +140,130 @@ __device__ __forceinline__ float ex2(float x) {
 // Contiguous tile range [lo, hi) of cluster c among n_clusters over all sequences' tiles.
 __device__ __forceinline__ int range_lo(long long c, long long total, long long nc) { return (int)((c * total) / nc); }
 
-// One warp: total tiles, this cluster's range, and the first sequence of the range.
+// The cluster whose contiguous range holds global tile t (ranges of empty clusters are skipped).
+__device__ __forceinline__ int cluster_of(long long t, long long total, long long nc) {
+  long long c = (t * nc) / (total > 0 ? total : 1);
+  if (c >= nc) c = nc - 1;
+  while (c + 1 < nc && range_lo(c + 1, total, nc) <= t) ++c;
+  while (c > 0 && range_lo(c, total, nc) > t) --c;
+  return (int)c;
+}
+
+__device__ __forceinline__ int seq_tiles(const Params& p, int b) { return tiles_of(clamp_len(p.lengths[b], p.n_max)); }
+
+// Tile counts of the first 256 sequences stay in registers (lane l holds sequences l + 32 k);
+// later ones are re-read from global memory.
+constexpr int kPlanRegs = 8;
+struct PlanTiles {
+  int t[kPlanRegs];
+  __device__ int at(const Params& p, int k, int lane) const {  // tiles of sequence 32 k + lane
+    if (k < kPlanRegs) {
+      int v = 0;
+#pragma unroll
+      for (int i = 0; i < kPlanRegs; ++i) v = (i == k) ? t[i] : v;
+      return v;
+    }
+    const int b = 32 * k + lane;
+    return b < p.B ? seq_tiles(p, b) : 0;
+  }
+};
+
+// Chunks of the chunked plan with chunk size c: the sum over sequences of ceil(tiles / c).
+__device__ int chunk_items(const Params& p, const PlanTiles& pt, int c, int lane) {
+  int n = 0;
+  const int nk = (p.B + 31) / 32;
+#pragma unroll
+  for (int k = 0; k < kPlanRegs; ++k)
+    if (k < nk) n += (pt.t[k] + c - 1) / c;
+  for (int k = kPlanRegs; k < nk; ++k) n += (pt.at(p, k, lane) + c - 1) / c;
+  return warp_sum_i(n);
+}
+
+// One warp: the work split.  Chunked plan when every non-empty sequence can have clusters of its
+// own and the smallest chunk that fits the clusters is within a quarter (or 4 tiles) of the
+// balanced share; else equal contiguous ranges over the concatenated tiles of all sequences.
 __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
+  PlanTiles pt;
   long long total = 0;
+  int maxt = 0, nonempty = 0;
   bool bad = false;
-  for (int b0 = 0; b0 < p.B; b0 += 32) {
-    const int b = b0 + lane;
+  const int nk = (p.B + 31) / 32;
+  for (int k = 0; k < nk; ++k) {
+    const int b = 32 * k + lane;
     int t = 0;
     if (b < p.B) {
       const int len = p.lengths[b];
       bad |= (len < 1 || len > p.n_max);
       t = tiles_of(clamp_len(len, p.n_max));
     }
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+#pragma unroll
+    for (int i = 0; i < kPlanRegs; ++i)
+      if (i == k) pt.t[i] = t;
+    maxt = max(maxt, t);
+    nonempty += t > 0 ? 1 : 0;
     total += t;
   }
-  if (__any_sync(0xffffffffu, bad) && lane == 0 && c == 0 && cluster_ctarank() == 0) raise_error(p.err, MLA_ERR_LENGTH);
-  const int lo = range_lo(c, total, p.n_clusters), hi = range_lo(c + 1, total, p.n_clusters);
-  int first_b = p.B, t_first = 0;
-  if (lo < hi) {
+#pragma unroll
+  for (int i = 0; i < kPlanRegs; ++i)
+    if (i >= nk) pt.t[i] = 0;
+  maxt = warp_max_i(maxt);
+  nonempty = warp_sum_i(nonempty);
+  {
+    long long v = total;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    total = v;
+  }
+  const bool any_bad = __any_sync(0xffffffffu, bad);
+  if (any_bad && lane == 0 && c == 0 && cluster_ctarank() == 0) raise_error(p.err, MLA_ERR_LENGTH);
+  const long long nc = p.n_clusters;
+  const int balanced = (int)((total + nc - 1) / nc);
+  int chunk = 0;
+  if (nonempty > 0 && nonempty <= nc) {
+    // chunk_items(maxt) = nonempty <= nc; below the balanced share it exceeds nc
+    int lo = max(1, min(balanced, maxt)), hi = maxt;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (chunk_items(p, pt, mid, lane) <= nc) hi = mid;
+      else lo = mid + 1;
+    }
+    if (lo <= balanced + max(4, balanced / 4)) chunk = lo;
+  }
+  int lo = 0, hi = 0, first_b = p.B, t_first = 0, item0 = 0, kb = 0;
+  if (chunk > 0) {
+    // cluster c takes chunk c: find its sequence by a scan of the chunk counts
+    int base_items = 0, base_tiles = 0;
+    for (int k = 0; k < nk && first_b == p.B; ++k) {
+      const int t = pt.at(p, k, lane);
+      const int kc = (t + chunk - 1) / chunk;
+      int ik = kc, it = t;  // inclusive prefix sums within the warp
+      for (int o = 1; o < 32; o <<= 1) {
+        const int vk = __shfl_up_sync(0xffffffffu, ik, o), vt = __shfl_up_sync(0xffffffffu, it, o);
+        if (lane >= o) {
+          ik += vk;
+          it += vt;
+        }
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, kc > 0 && base_items + ik > c);
+      if (m) {
+        const int l0 = __ffs(m) - 1;
+        const int kk = __shfl_sync(0xffffffffu, kc, l0), tt = __shfl_sync(0xffffffffu, t, l0);
+        item0 = base_items + __shfl_sync(0xffffffffu, ik, l0) - kk;
+        t_first = base_tiles + __shfl_sync(0xffffffffu, it, l0) - tt;
+        first_b = 32 * k + l0;
+        kb = kk;
+        const int j = c - item0;
+        lo = t_first + j * chunk;
+        hi = t_first + min((j + 1) * chunk, tt);
+      }
+      base_items += __shfl_sync(0xffffffffu, ik, 31);
+      base_tiles += __shfl_sync(0xffffffffu, it, 31);
+    }
+  } else {
+    lo = range_lo(c, total, nc);
+    hi = range_lo(c + 1, total, nc);
+  }
+  if (chunk == 0 && lo < hi) {
     int base = 0;  // tiles before batch b0
     for (int b0 = 0; b0 < p.B && first_b == p.B; b0 += 32) {
       const int b = b0 + lane;
@@ -151,6 +288,11 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
     sm.hi = hi;
     sm.b0 = first_b;
     sm.t_b0 = t_first;
+    sm.chunk = chunk;
+    sm.item0 = item0;
+    sm.kb = kb;
+    sm.total = total;
+    sm.bad = any_bad ? 1 : 0;
   }
 }
 
@@ -161,8 +303,9 @@ struct SegIter {
   int n_max, B;
   __device__ SegIter(const Smem& sm, const Params& p) : b(sm.b0), tb(sm.t_b0), t(sm.lo), hi(sm.hi),
                                                         lengths(p.lengths), n_max(p.n_max), B(p.B) {}
-  // On success: sequence b, tiles [begin, end) of it, its length, whether the range holds all of it.
-  __device__ bool next(int& sb, int& begin, int& end, int& len, bool& whole) {
+  // On success: sequence b, tiles [begin, end) of it, its length, whether the range holds all of it,
+  // and the global index of its first tile.
+  __device__ bool next(int& sb, int& begin, int& end, int& len, bool& whole, int& base) {
     while (t < hi && b < B) {
       len = clamp_len(lengths[b], n_max);
       const int nt = tiles_of(len);
@@ -172,6 +315,7 @@ struct SegIter {
         continue;
       }
       sb = b;
+      base = tb;
       begin = t - tb;
       end = min(hi, tb + nt) - tb;
       whole = (begin == 0 && end == nt);
@@ -184,6 +328,46 @@ struct SegIter {
   }
 };
 
+// Partial slots of sequence b (first global tile `base`, nt tiles): slot 2c holds the partial of
+// cluster c's first segment, slot 2c + 1 that of its last segment.
+__device__ int list_slots(const Params& p, Smem& sm, int base, int nt) {
+  int n = 0;
+  if (sm.chunk > 0) {
+    for (int k = 0; k < sm.kb && n < kMaxClusters; ++k) sm.slots[n++] = (int16_t)(2 * (sm.item0 + k));
+  } else {
+    const long long total = sm.total, nc = p.n_clusters;
+    const int c0 = cluster_of(base, total, nc), c1 = cluster_of((long long)base + nt - 1, total, nc);
+    for (int c = c0; c <= c1 && n < kMaxClusters; ++c) {
+      const long long lo = range_lo(c, total, nc), hi = range_lo(c + 1, total, nc);
+      if (hi > lo) sm.slots[n++] = (int16_t)(2 * c + (lo >= base ? 0 : 1));
+    }
+  }
+  sm.nslots = n;
+  return n;
+}
+
+// Counts this CTA's arrival for (sequence, latent half) and reports whether it was the last of
+// `expected`.  The counter holds (epoch << 8) | arrivals; a value from another launch (another
+// epoch, or the 0 the last arrival leaves behind) counts as no arrival, so the workspace needs no
+// initialisation.  Every failed compare-and-swap means another CTA's arrival succeeded, so the
+// loop ends after at most `expected` rounds; the bound is only a guard.
+__device__ bool arrive_last(unsigned long long* ctr, unsigned long long epoch, int expected, int32_t* err) {
+  unsigned long long cur = 0;  // the value the previous launch's last arrival leaves
+  for (int i = 0; i < 4096; ++i) {
+    const unsigned long long base = (cur >> 8) == epoch ? cur : (epoch << 8);
+    const unsigned long long next = base + 1;
+    const unsigned long long prev = atomicCAS(ctr, cur, next);
+    if (prev == cur) {
+      if ((int)(next & 255ull) < expected) return false;
+      atomicExch(ctr, 0ull);  // every arrival of this launch is in: leave the counter for the next one
+      return true;
+    }
+    cur = prev;
+  }
+  raise_error(err, MLA_ERR_TIMEOUT);
+  return false;
+}
+
 __device__ __forceinline__ void fail_timeout(Smem& sm, int32_t* err) {
   raise_error(err, MLA_ERR_TIMEOUT);
   sm.abort = 1;
@@ -194,8 +378,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
-  uint8_t* xbuf = smem + kStages * kStageBytes;  // 2 receive + 2 staging exchange buffers
-  Smem& sm = *reinterpret_cast<Smem*>(smem + kStages * kStageBytes + 4 * kXBytes);
+  uint8_t* xbuf = smem + kXOff;        // 2 receive + 2 staging exchange buffers (first: the query)
+  uint8_t* qrope = smem + kQRopeOff;    // rotary half of the first query
+  Smem& sm = *reinterpret_cast<Smem*>(smem + kSmemOff);
   volatile int* abort_flag = &sm.abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -208,6 +393,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     // softmax-side arrivals are one per softmax warp, after a __syncwarp
+    mbar_init(smem_u32(&sm.q_tma), 1);
     mbar_init(smem_u32(&sm.q_full), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.s_empty), 4);  // the four exchange warps
@@ -216,16 +402,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&sm.drain), 2);  // one commit from each MMA-issuing thread
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.x_full[i]), 1);  // 1 local arrive.expect_tx + the peer's st.async bytes
-      mbar_init(smem_u32(&sm.x_free[i]), 1);  // 1 remote arrive from the peer
+      // 1 remote arrive from the peer: first when the peer has copied its query out of its exchange
+      // buffers, then each time it has read a partial this CTA sent
+      mbar_init(smem_u32(&sm.x_free[i]), 1);
       mbar_init(smem_u32(&sm.own_ready[i]), 4);
       mbar_init(smem_u32(&sm.stg_free[i]), kSoftmaxWarps);
       for (int q = 0; q < 4; ++q) mbar_init(smem_u32(&sm.red_bar[i][q]), 2);
     }
     mbar_init(smem_u32(&sm.sum_bar), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.pub_bar), kSoftmaxWarps);
+    mbar_init(smem_u32(&sm.last_bar), 1);
     sm.abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&p.tm_ckv);
     prefetch_tensormap(&p.tm_kr);
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_qp);
   }
   if (warp == 0) plan_range(p, cl, sm, lane);
   if (warp == 1) {
@@ -237,18 +429,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_after();
   cluster_sync();  // the peer's barriers are initialised before any remote arrive
   const uint32_t tmem = sm.tmem_base;
-  if (threadIdx.x == 0 && rank == 0) p.ws_plan[cl] = sm.b0;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol = policy_evict_first();
       SegIter seg(sm, p);
-      int b, begin, end, len;
+      int b, begin, end, len, base;
       bool whole;
       uint32_t it = 0;
-      bool ok = true;
-      while (ok && seg.next(b, begin, end, len, whole)) {
+      bool ok = true, q_issued = false;
+      while (ok && seg.next(b, begin, end, len, whole, base)) {
+        if (!q_issued) {
+          // the first sequence's query (this CTA's halves) goes in ahead of the cache tiles: latent
+          // half into the four exchange buffers (free until the first exchange), rotary half apart
+          const uint32_t qb = smem_u32(&sm.q_tma);
+          mbar_arrive_expect_tx(qb, kQLatBytes + kQRopeBytes);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            tma_load_2d(smem_u32(xbuf + j * kXBytes), &p.tm_q, qb, 256 * (int)rank + 64 * j, b * kNH, pol);
+          tma_load_2d(smem_u32(qrope), &p.tm_qp, qb, 32 * (int)rank, b * kNH, pol);
+          q_issued = true;
+        }
         for (int i = begin; i < end && ok; ++i, ++it) {
           const uint32_t st = it % kStages, ph = (it / kStages) & 1u;
           if (!mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
@@ -269,6 +471,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0;
       for (uint32_t k = first; k < it; ++k)
         mbar_wait(smem_u32(&sm.full[k % kStages]), (k / kStages) & 1u, abort_flag, kWaitLimitNs);
+      if (q_issued) mbar_wait(smem_u32(&sm.q_tma), 0, abort_flag, kWaitLimitNs);
+    }
+    // lengths outside [1, n_max] (an error already flagged): sequences left without tiles get a
+    // zero context and lse = -inf from cluster 0, each CTA its latent half
+    if (cl == 0 && sm.bad) {
+      for (int b = 0; b < p.B; ++b) {
+        if (seq_tiles(p, b) != 0) continue;
+        for (int i = lane; i < kNH * 32; i += 32)
+          reinterpret_cast<uint4*>(p.ctx + ((int64_t)b * kNH + (i >> 5)) * kDC + 256 * rank)[i & 31] =
+              make_uint4(0, 0, 0, 0);
+        if (rank == 0 && p.lse != nullptr)
+          for (int hh = lane; hh < kNH; hh += 32) p.lse[(int64_t)b * kNH + hh] = -INFINITY;
+      }
     }
   } else if (warp == 1 || warp == kPvWarp) {
     // ------------------------------------------------------------------ MMA issuers
@@ -280,7 +495,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     const uint32_t idesc_pv = idesc_bf16_f32(128, 256, 0, 1);
     const uint32_t tO = tmem + kColO, tS = tmem + kColS, tP = tmem + kColP, tQ = tmem + kColQ;
     SegIter seg(sm, p);
-    int b, begin, end, len;
+    int b, begin, end, len, base;
     bool whole;
     uint32_t it = 0, nseg = 0;  // it: global index of the next tile
     bool ok = true;
@@ -347,7 +562,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
-    while (ok && seg.next(b, begin, end, len, whole)) {
+    while (ok && seg.next(b, begin, end, len, whole, base)) {
       if (is_qk) {
         if (!wait_or_fail(smem_u32(&sm.q_full), nseg & 1u, false)) break;
         tc_fence_after();
@@ -405,9 +620,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&sm.s_empty));
-      // staging xi is free once the peer consumed tile t - 2 (so its copy is done) and this CTA's
-      // softmax warps have read it
-      if (!wait_or_fail(smem_u32(&sm.x_free[xi]), (use & 1u) ^ 1u, true)) break;
+      // the peer's receive buffer xi is free once the peer has copied its query out (phase 0) and
+      // read this CTA's tile t - 2 (phase use); staging xi once this CTA's softmax warps read it
+      if (!wait_or_fail(smem_u32(&sm.x_free[xi]), use & 1u, true)) break;
       if (!wait_or_fail(smem_u32(&sm.stg_free[xi]), (use & 1u) ^ 1u, false)) break;
       // The softmax warps release staging xi only after they have waited for receive buffer xi of
       // tile t - 2, so that phase of x_full[xi] is complete and this tile's expected byte count
@@ -447,10 +662,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar);
     };
     SegIter seg(sm, p);
-    int b, begin, end, len;
+    int b, begin, end, len, base;
     bool whole;
     uint32_t tb = 0;           // global tile counter
-    uint32_t nseg = 0;
+    uint32_t nseg = 0, npart = 0;
     bool ok = true;
     bool first_seg = true;     // the first segment of the range uses partial slot 2c, the last 2c + 1
     auto wait_or_fail = [&](uint32_t bar, uint32_t par, bool cl_scope) {
@@ -462,9 +677,47 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       return ok;
     };
-    while (ok && seg.next(b, begin, end, len, whole)) {
+    while (ok && seg.next(b, begin, end, len, whole, base)) {
       // ---- this sequence's query half into TMEM (A operand of the score MMA)
-      {
+      if (nseg == 0) {
+        // staged by TMA: latent chunk c = box c of the exchange buffers (128-byte swizzle, 128-byte
+        // rows), rotary half in its own buffer (64-byte swizzle, 64-byte rows)
+        if (!wait_or_fail(smem_u32(&sm.q_tma), 0, false)) break;
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = 2 * half + cc;
+          const uint32_t row = xb + c * kXBytes + h * 128;
+          uint32_t r[32];
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 u = ld_shared_v4_b32(row + ((v ^ (h & 7)) << 4));
+            r[4 * v] = u.x; r[4 * v + 1] = u.y; r[4 * v + 2] = u.z; r[4 * v + 3] = u.w;
+          }
+          tmem_st32(tQ + c * 32, r);
+        }
+        if (half == 1) {
+          const uint32_t row = smem_u32(qrope) + h * 64;
+          uint32_t r16[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint4 u = ld_shared_v4_b32(row + ((v ^ ((h >> 1) & 3)) << 4));
+            r16[4 * v] = u.x; r16[4 * v + 1] = u.y; r16[4 * v + 2] = u.z; r16[4 * v + 3] = u.w;
+          }
+          tmem_st16(tQ + 128, r16);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        warp_arrive(smem_u32(&sm.q_full));
+        if (sw == 0 && lane == 0) {
+          // every softmax warp has copied its rows out: the peer may now write this CTA's buffers
+          if (mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, kWaitLimitNs)) {
+            mbar_arrive_remote(x_free_peer0);
+            mbar_arrive_remote(x_free_peer0 + 8);
+          } else {
+            fail_timeout(sm, p.err);
+          }
+        }
+      } else {
         const __nv_bfloat16* qt = p.q_tilde + ((int64_t)b * kNH + h) * p.ldqt + 256 * rank;
         const __nv_bfloat16* qp = p.q_pe + ((int64_t)b * kNH + h) * p.ldqp + 32 * rank;
 #pragma unroll
@@ -608,18 +861,86 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (rank == 0 && half == 0 && p.lse != nullptr)
           p.lse[(int64_t)b * kNH + h] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
       } else {
-        const int slot = 2 * cl + (first_seg ? 0 : 1);
-        float* out = p.ws_o + (((int64_t)slot * 2 + rank) * kNH + h) * 256 + 128 * half;
+        // ---- partial: publish (O, m, l) in this segment's slot; the last of the sequence's
+        // clusters to arrive (per latent half) merges every partial into ctx
+        const int own = 2 * cl + (first_seg ? 0 : 1);
+        float* out = p.ws_o + (((int64_t)own * 2 + rank) * 256 + 128 * half) * kNH + h;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
           tmem_ld32(tO + c * 32, r);
           tmem_ld_wait();
-          uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
-          for (int v = 0; v < 8; ++v) dst[v] = make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+          for (int k = 0; k < 32; ++k) out[(c * 32 + k) * kNH] = __uint_as_float(r[k]);
         }
-        if (rank == 0 && half == 0) p.ws_ml[(int64_t)slot * kNH + h] = make_float2(m_run, l_tot);
+        if (half == 0) p.ws_ml[((int64_t)own * 2 + rank) * kNH + h] = make_float2(m_run, l_tot);
+        __threadfence();
+        warp_arrive(smem_u32(&sm.pub_bar));
+        if (sw == 0 && lane == 0) {
+          bool last = false;
+          if (mbar_wait(smem_u32(&sm.pub_bar), npart & 1u, abort_flag, kWaitLimitNs)) {
+            const int ns = list_slots(p, sm, base, tiles_of(len));
+            __threadfence();
+            last = arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err);
+            if (last) __threadfence();
+          } else {
+            fail_timeout(sm, p.err);
+          }
+          sm.is_last = last ? 1 : 0;
+          mbar_arrive(smem_u32(&sm.last_bar));
+        }
+        if (!wait_or_fail(smem_u32(&sm.last_bar), npart & 1u, false)) break;
+        ++npart;
+        if (sm.is_last) {
+          __threadfence();
+          // the other partials come from other SMs: read them through L2 (ld.global.cg).  Every
+          // sum runs in slot order with this CTA's own partial (kept in TMEM) in its slot's place,
+          // so the result does not depend on which cluster arrived last.
+          const int ns = sm.nslots;
+          auto ml_of = [&](int sl) {
+            return sl == own ? make_float2(m_run, l_tot) : __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
+          };
+          float M = -INFINITY;
+          for (int i = 0; i < ns; ++i) M = fmaxf(M, ml_of(sm.slots[i]).x);
+          float L = 0.f;
+          for (int i = 0; i < ns; ++i) {
+            const float2 ml = ml_of(sm.slots[i]);
+            L += ml.y * ex2(ml.x - M);
+          }
+          const float inv = 1.f / L;
+          __nv_bfloat16* dst = p.ctx + ((int64_t)b * kNH + h) * kDC + 256 * rank + 128 * half;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_ld_wait();
+            float acc[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+            for (int i = 0; i < ns; ++i) {
+              const int sl = sm.slots[i];
+              const float w = ex2(ml_of(sl).x - M) * inv;
+              if (sl == own) {
+#pragma unroll
+                for (int k = 0; k < 32; ++k) acc[k] = fmaf(w, __uint_as_float(r[k]), acc[k]);
+              } else {
+                const float* src = p.ws_o + (((int64_t)sl * 2 + rank) * 256 + 128 * half + c * 32) * kNH + h;
+                float o[32];
+#pragma unroll
+                for (int k = 0; k < 32; ++k) o[k] = __ldcg(src + k * kNH);
+#pragma unroll
+                for (int k = 0; k < 32; ++k) acc[k] = fmaf(w, o[k], acc[k]);
+              }
+            }
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                                 pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+          }
+          if (rank == 0 && half == 0 && p.lse != nullptr)
+            p.lse[(int64_t)b * kNH + h] = (M + log2f(L)) * 0.69314718055994531f;
+        }
       }
       first_seg = false;
       ++nseg;
@@ -635,101 +956,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------------------------------
-// Combine: merge the fp32 partials of sequences whose tiles span several clusters
-// ------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) combine_kernel(const __grid_constant__ Params p) {
-  const int b = blockIdx.x;
-  const int h0 = blockIdx.y * 8;
-  __shared__ int s_info[4];  // c_lo, c_hi, tiles of b, total tiles
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
-    long long total = 0, before = 0;
-    for (int b0 = 0; b0 < p.B; b0 += 32) {
-      const int bb = b0 + lane;
-      int t = bb < p.B ? tiles_of(clamp_len(p.lengths[bb], p.n_max)) : 0;
-      int tb = bb < b ? t : 0;
-      for (int o = 16; o > 0; o >>= 1) {
-        t += __shfl_xor_sync(0xffffffffu, t, o);
-        tb += __shfl_xor_sync(0xffffffffu, tb, o);
-      }
-      total += t;
-      before += tb;
-    }
-    if (lane == 0) {
-      const int nt = tiles_of(clamp_len(p.lengths[b], p.n_max));
-      const long long nc = p.n_clusters;
-      auto cluster_of = [&](long long t) {
-        long long c = (t * nc) / (total > 0 ? total : 1);
-        while (c + 1 < nc && range_lo(c + 1, total, nc) <= t) ++c;
-        while (c > 0 && range_lo(c, total, nc) > t) --c;
-        return (int)c;
-      };
-      s_info[2] = nt;
-      s_info[3] = (int)total;
-      s_info[0] = nt > 0 ? cluster_of(before) : 0;
-      s_info[1] = nt > 0 ? cluster_of(before + nt - 1) : 0;
-    }
-  }
-  __syncthreads();
-  const int c_lo = s_info[0], c_hi = s_info[1], nt = s_info[2];
-  if (nt == 0) {  // empty sequence: zero context, lse = -inf
-    for (int i = threadIdx.x; i < 8 * kDC; i += blockDim.x)
-      p.ctx[((int64_t)b * kNH + h0 + i / kDC) * kDC + i % kDC] = __float2bfloat16_rn(0.f);
-    if (p.lse && threadIdx.x < 8) p.lse[(int64_t)b * kNH + h0 + threadIdx.x] = -INFINITY;
-    return;
-  }
-  if (c_lo == c_hi) return;  // one cluster held the whole sequence and wrote ctx itself
-  // ---- the partial slots of this sequence, resolved once (clusters with an empty range hold none)
-  constexpr int kMaxSlots = 256;
-  __shared__ int s_slot[kMaxSlots];
-  __shared__ int s_nslot;
-  __shared__ float s_w[8][kMaxSlots];  // per head: e^{m_s - M} / L, the weight of partial s
-  if (threadIdx.x == 0) {
-    const long long total = s_info[3], nc = p.n_clusters;
-    int ns = 0;
-    long long lo = range_lo(c_lo, total, nc);
-    for (int c = c_lo; c <= c_hi && ns < kMaxSlots; ++c) {
-      const long long hi = range_lo(c + 1, total, nc);
-      if (hi > lo) s_slot[ns++] = 2 * c + (p.ws_plan[c] == b ? 0 : 1);
-      lo = hi;
-    }
-    s_nslot = ns;
-  }
-  __syncthreads();
-  const int ns = s_nslot;
-  {  // one warp per head: running-max merge of (m_s, l_s)
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, hh = h0 + warp;
-    float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, p.ws_ml[(int64_t)s_slot[s] * kNH + hh].x);
-    M = warp_max(M);
-    float L = 0.f;
-    for (int s = lane; s < ns; s += 32) {
-      const float2 ml = p.ws_ml[(int64_t)s_slot[s] * kNH + hh];
-      const float w = ex2(ml.x - M);
-      s_w[warp][s] = w;
-      L += w * ml.y;
-    }
-    L = warp_sum(L);
-    const float inv = 1.f / L;
-    for (int s = lane; s < ns; s += 32) s_w[warp][s] *= inv;
-    if (lane == 0 && p.lse) p.lse[(int64_t)b * kNH + hh] = (M + log2f(L)) * 0.69314718055994531f;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 8 * (kDC / 4); i += blockDim.x) {
-    const int hl = i / (kDC / 4), hh = h0 + hl, d = (i % (kDC / 4)) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < ns; ++s) {
-      const float w = s_w[hl][s];
-      const float4 o = *reinterpret_cast<const float4*>(
-          p.ws_o + (((int64_t)s_slot[s] * 2 + (d >> 8)) * kNH + hh) * 256 + (d & 255));
-      acc.x += w * o.x; acc.y += w * o.y; acc.z += w * o.z; acc.w += w * o.w;
-    }
-    __nv_bfloat16* out = p.ctx + ((int64_t)b * kNH + hh) * kDC + d;
-    *reinterpret_cast<uint2*>(out) = make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
-  }
-}
-
-// ------------------------------------------------------------------------------------------
 // Host side
 // ------------------------------------------------------------------------------------------
 bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint64_t s1_bytes,
@@ -740,14 +966,31 @@ bool make_map_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
   return make_tensor_map_bf16(m, base, 3, dims, strides, box, sw);
 }
 
-size_t smem_bytes() { return (size_t)kStages * kStageBytes + 4 * kXBytes + sizeof(Smem) + 1024; }
+size_t smem_bytes() { return (size_t)kSmemOff + sizeof(Smem) + 1024; }
+static_assert(kSmemOff + sizeof(Smem) + 1024 <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
+
+// Workspace layout for n_clusters clusters and B sequences: partial O, partial (m, l), counters.
+size_t ws_o_bytes(size_t nc) { return 2 * nc * 2 * 128 * 256 * sizeof(float); }
+size_t ws_ml_bytes(size_t nc) { return 2 * nc * 2 * 128 * sizeof(float2); }
+size_t ws_bytes(size_t nc, size_t B) { return ws_o_bytes(nc) + ws_ml_bytes(nc) + B * 2 * sizeof(unsigned long long) + 256; }
+
+// A launch identifier for the arrival counters: unique within the process (a 56-bit counter
+// started from the clock), never 0.
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> counter{
+      (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count() * 0x9E3779B97F4A7C15ull};
+  unsigned long long e = 0;
+  while (e == 0) e = counter.fetch_add(1, std::memory_order_relaxed) & ((1ull << 56) - 1);
+  return e;
+}
 
 // Upper bound of clusters: one CTA pair per two SMs (sizes the workspace).
 int max_clusters() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms / 2 > 0 ? sms / 2 : 1;
+  const int n = sms / 2 < kMaxClusters ? sms / 2 : kMaxClusters;
+  return n > 0 ? n : 1;
 }
 
 // Clusters that can be resident at once (GPCs with an odd number of free SMs cannot host a full
@@ -776,11 +1019,7 @@ int num_clusters() {
 
 }  // namespace decode_tc
 
-size_t decode_tc_workspace(int B) {
-  (void)B;
-  const size_t nc = decode_tc::max_clusters();
-  return 2 * nc * (2 * 128 * 256 * sizeof(float)) + 2 * nc * 128 * sizeof(float2) + nc * sizeof(int32_t) + 1024;
-}
+size_t decode_tc_workspace(int B) { return decode_tc::ws_bytes(decode_tc::max_clusters(), B > 0 ? B : 0); }
 
 cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   using namespace decode_tc;
@@ -794,6 +1033,14 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
       !make_map_3d(&p.tm_kr, a.k_r, kDR, a.n_max, a.B, (uint64_t)a.kr_r * 2, bstride_r, 32, kTile,
                    CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
+  {
+    const uint64_t qd[2] = {(uint64_t)kDC, (uint64_t)a.B * kNH}, qs[1] = {(uint64_t)a.ldqt * 2};
+    const uint64_t rd[2] = {(uint64_t)kDR, (uint64_t)a.B * kNH}, rs[1] = {(uint64_t)a.ldqp * 2};
+    const uint32_t qbox[2] = {64, kNH}, rbox[2] = {32, kNH};
+    if (!make_tensor_map_bf16(&p.tm_q, a.q_tilde, 2, qd, qs, qbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_tensor_map_bf16(&p.tm_qp, a.q_pe, 2, rd, rs, rbox, CU_TENSOR_MAP_SWIZZLE_64B))
+      return cudaErrorInvalidValue;
+  }
   p.q_tilde = static_cast<const __nv_bfloat16*>(a.q_tilde);
   p.ldqt = a.ldqt;
   p.q_pe = static_cast<const __nv_bfloat16*>(a.q_pe);
@@ -807,19 +1054,17 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   p.lse = a.lse;
   uint8_t* w = static_cast<uint8_t*>(ws);
   p.ws_o = reinterpret_cast<float*>(w);
-  w += 2 * (size_t)nc * (2 * 128 * 256 * sizeof(float));
+  w += ws_o_bytes(nc);
   p.ws_ml = reinterpret_cast<float2*>(w);
-  w += 2 * (size_t)nc * 128 * sizeof(float2);
-  p.ws_plan = reinterpret_cast<int32_t*>(w);
+  w += ws_ml_bytes(nc);
+  p.ws_ctr = reinterpret_cast<unsigned long long*>(w);
+  p.epoch = next_epoch();
   p.err = a.err;
 
   const size_t smem = smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   decode_kernel<<<2 * nc, kThreads, smem, st>>>(p);
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  combine_kernel<<<dim3(a.B, kNH / 8), 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -831,13 +1076,15 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
 // budget), code issuing work while a stream is being captured into a CUDA graph, or a caller that
 // only holds pointers handed to it by someone else.  For them the split-KV scratch lives in this
 // file-scope array, which every GPU that loads the library holds until the process exits.
-// Sized for 74 clusters (one CTA pair per two SMs of a 148-SM B200): 74 x 2 partial slots of
-// 128 heads x 512 fp32 features, their (m, l) pairs and the per-cluster plan, about 37.1 MiB.
+// Sized for 74 clusters (one CTA pair per two SMs of a 148-SM B200) and up to 4096 sequences:
+// 74 x 2 partial slots of 128 heads x 512 fp32 features, their (m, l) pairs and two arrival
+// counters per sequence, about 37.2 MiB.
 namespace {
 constexpr size_t kStaticMaxClusters = 74;
-constexpr size_t kStaticScratchBytes = 2 * kStaticMaxClusters * (2 * 128 * 256 * sizeof(float)) +
-                                       2 * kStaticMaxClusters * 128 * sizeof(float2) +
-                                       kStaticMaxClusters * sizeof(int32_t) + 1024;
+constexpr size_t kStaticMaxBatch = 4096;
+constexpr size_t kStaticScratchBytes = 2 * kStaticMaxClusters * 2 * 128 * 256 * sizeof(float) +
+                                       2 * kStaticMaxClusters * 2 * 128 * sizeof(float2) +
+                                       kStaticMaxBatch * 2 * sizeof(unsigned long long) + 256;
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 }  // namespace
 

@@ -117,7 +117,7 @@ size_t mla_decode_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int3
 int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
   if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
   const int cap = topk > 0 ? topk : n_max;
-  if (dtype == MLA_BF16 && topk == 0) return 2;  // tensor-core decode + combine
+  if (dtype == MLA_BF16 && topk == 0) return 1;  // tensor-core decode, partials merged in-kernel
   return mla::decode_simt_splits(B, cap) > 1 ? 2 : 1;
 }
 
@@ -148,6 +148,8 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B, const vo
   MLA_TRY(check_bf16_stride(dtype, ckv_rstride, "ckv_rstride"));
   MLA_TRY(check_bf16_stride(dtype, kr_bstride, "kr_bstride"));
   MLA_TRY(check_bf16_stride(dtype, kr_rstride, "kr_rstride"));
+  if (dtype == MLA_BF16 && !topk_idx && (int64_t)B * ((n_max + 63) / 64) >= ((int64_t)1 << 31))
+    return fail(MLA_ERR_UNSUPPORTED, "B * ceil(n_max / 64) must stay below 2^31");
   const size_t need = mla_decode_workspace_size(dims, dtype, B, n_max, topk_idx ? topk : 0);
   if (!workspace || ws_bytes < need)
     return fail(MLA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace ? ws_bytes : (size_t)0);
@@ -186,8 +188,8 @@ mla_status mla_decode_absorb_static(mla_dims dims, mla_dtype dtype, int32_t B, c
   const size_t have = mla::decode_static_scratch_bytes();
   if (need > have)
     return fail(MLA_ERR_WORKSPACE,
-                "mla_decode_absorb_static: this device needs %zu bytes of split-KV scratch, the built-in "
-                "scratch holds %zu (it is sized for up to 148 SMs)", need, have);
+                "mla_decode_absorb_static: this call needs %zu bytes of split-KV scratch, the built-in "
+                "scratch holds %zu (it is sized for up to 148 SMs and 4096 sequences)", need, have);
   void* scratch = nullptr;
   MLA_TRY(cuda_status(mla::decode_static_scratch(&scratch), "mla_decode_absorb_static scratch set-up"));
   return mla_decode_absorb(dims, dtype, B, q_tilde, ldqt, q_pe, ldqp, c_kv, ckv_bstride, ckv_rstride, k_r,
