@@ -180,21 +180,48 @@ def run_ours(args, rank, world, local_rank):
     stream = torch.cuda.current_stream(dev)
     n_launch = 2 + api.mla_decode_num_launches(dims, torch.bfloat16, B, cfg.n_max)
 
-    def step(qn, qp):
-        api.mla_absorb_q(dims, qn, w, q_tilde, stream=stream)
-        ev[1].record(stream)
+    def step_on(st, qn, qp, marks=False):
+        api.mla_absorb_q(dims, qn, w, q_tilde, stream=st)
+        if marks:
+            ev[1].record(st)
         api.mla_decode_absorb(dims, q_tilde, qp, c_kv, k_r, lengths, cfg.scale, ctx=ctx, lse=lse, workspace=ws,
-                              dev_err=err, stream=stream)
-        ev[2].record(stream)
-        api.mla_out_up(dims, ctx, w, out, stream=stream)
+                              dev_err=err, stream=st)
+        if marks:
+            ev[2].record(st)
+        api.mla_out_up(dims, ctx, w, out, stream=st)
 
-    # ---- device-resident timing ------------------------------------------------------------
+    def step(qn, qp):
+        step_on(stream, qn, qp, marks=True)
+
+    # ---- per-call timing (each call launched on its own, events between the calls) ------------
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K + args.warmup)]
-    for i in range(args.warmup):
+    for i in range(args.warmup + K):
         ev = evs[i]
         flush.zero_()
         ev[0].record(stream); step(q_nope, q_pe); ev[3].record(stream)
+    torch.cuda.synchronize()
+    per = {"absorb_q": [], "decode": [], "out_up": []}
+    for ev in evs[args.warmup:]:
+        per["absorb_q"].append(ev[0].elapsed_time(ev[1]))
+        per["decode"].append(ev[1].elapsed_time(ev[2]))
+        per["out_up"].append(ev[2].elapsed_time(ev[3]))
+    ms = {k: statistics.mean(v) for k, v in per.items()}
+
+    # ---- the step as a server runs it: the three calls captured once in a CUDA graph and
+    # replayed (no host work between the kernels); CUDA events around every replay --------------
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            step_on(cap, q_nope, q_pe)
+    stream.wait_stream(cap)
+    torch.cuda.synchronize()
+    gev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K + args.warmup)]
+    for i in range(args.warmup):
+        flush.zero_()
+        gev[i][0].record(stream); graph.replay(); gev[i][1].record(stream)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -202,21 +229,14 @@ def run_ours(args, rank, world, local_rank):
     with ClockSampler(local_rank) as clk:
         t_wall = time.perf_counter()
         for i in range(args.warmup, args.warmup + K):
-            ev = evs[i]
             flush.zero_()
-            ev[0].record(stream); step(q_nope, q_pe); ev[3].record(stream)
+            gev[i][0].record(stream); graph.replay(); gev[i][1].record(stream)
         torch.cuda.synchronize()
         t_wall = time.perf_counter() - t_wall
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    per = {"step": [], "absorb_q": [], "decode": [], "out_up": []}
-    for ev in evs[args.warmup:]:
-        per["step"].append(ev[0].elapsed_time(ev[3]))
-        per["absorb_q"].append(ev[0].elapsed_time(ev[1]))
-        per["decode"].append(ev[1].elapsed_time(ev[2]))
-        per["out_up"].append(ev[2].elapsed_time(ev[3]))
-    ms = {k: statistics.mean(v) for k, v in per.items()}
+    ms["step"] = statistics.mean(e[0].elapsed_time(e[1]) for e in gev[args.warmup:])
     assert api.mla_get_device_error(err) == 0, "device error flag raised during the bench"
 
     # ---- end to end through the public API with host buffers ---------------------------------
@@ -262,7 +282,9 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": cfg.name, "B_per_gpu": B, "n_max": cfg.n_max, "n_h": cfg.n_h, "d_c": cfg.d_c,
                    "d_r": cfg.d_r, "d_h": cfg.d_h, "d_v": cfg.d_v, "global_batch": world * B,
                    "parallelism": f"batch-sharded replicas x{world}", "l2": "flushed (256 MiB write) before each step",
-                   "timing": "CUDA events around each step, mean over steps, max over ranks"},
+                   "timing": "CUDA events around each replay of the step's CUDA graph (the three calls "
+                             "captured once), mean over steps, max over ranks; per-call times from separate "
+                             "launches with events between the calls"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mla_decode_absorb",
                      "peak_source": peaks["source"] + " (hbm_gbs, burst)",

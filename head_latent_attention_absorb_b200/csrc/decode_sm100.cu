@@ -88,10 +88,11 @@ struct Params {
   float scale_log2;
   __nv_bfloat16* ctx;
   float* lse;
-  float* ws_o;     // [2 n_clusters slots][2 halves][256 features][128 heads] fp32, unnormalised
-                   // (feature-major, so a warp's 32 heads of one feature are 128 contiguous bytes)
+  float* ws_o;     // [2 n_clusters slots][2 halves][128 heads][256 features] bf16 partial contexts,
+                   // each normalised by its own softmax sum (16-byte chunks rotated by head & 15)
   float2* ws_ml;   // [2 n_clusters slots][2 halves][128] (running max in log2 units, sum)
   unsigned long long* ws_ctr;  // [B][2 halves] arrival counters: (epoch << 8) | arrivals
+  unsigned long long* ws_ready;  // [2 n_clusters slots][2 halves] partial published: the writer's epoch
   unsigned long long epoch;    // unique per launch, never 0, < 2^56
   int32_t* err;
 };
@@ -103,6 +104,7 @@ struct Smem {
   uint64_t own_ready[2], stg_free[2];  // this CTA's fp16 partial staged / read by the softmax warps
   uint64_t red_bar[2][4], sum_bar; // row-max rendezvous of the two warps of a lane quadrant / final sum
   uint64_t pub_bar, last_bar;      // partial published by all softmax warps / merge decision made
+  uint64_t mrg_full;               // the other cluster's partial bulk-loaded for the merge
   float red[2][2][kNH];            // [tile parity][key half][head] partial row max
   float lsum[2][kNH];              // [key half][head] partial softmax sum
   int16_t slots[kMaxClusters];     // partial slots of the sequence being merged
@@ -136,6 +138,10 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// bf16 halves of a packed pair, widened exactly to fp32 (low half = first element).
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
 // Contiguous tile range [lo, hi) of cluster c among n_clusters over all sequences' tiles.
 __device__ __forceinline__ int range_lo(long long c, long long total, long long nc) { return (int)((c * total) / nc); }
@@ -227,7 +233,10 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
       if (chunk_items(p, pt, mid, lane) <= nc) hi = mid;
       else lo = mid + 1;
     }
-    if (lo <= balanced + max(4, balanced / 4)) chunk = lo;
+    // One tile longer than the smallest fitting chunk (never more chunks, since chunk_items only
+    // falls as the chunk grows): a split sequence's last chunk is then shorter than the others, so
+    // its cluster finishes first and publishes its partial while the merging cluster still works.
+    if (lo <= balanced + max(4, balanced / 4)) chunk = (lo > 1 && lo < maxt) ? lo + 1 : lo;
   }
   int lo = 0, hi = 0, first_b = p.B, t_first = 0, item0 = 0, kb = 0;
   if (chunk > 0) {
@@ -373,6 +382,23 @@ __device__ __forceinline__ void fail_timeout(Smem& sm, int32_t* err) {
   sm.abort = 1;
 }
 
+__device__ __forceinline__ void st_release_gpu(unsigned long long* f, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(f), "l"(v) : "memory");
+}
+
+// Bounded wait until *f == want (acquire at GPU scope); false on abort or after kWaitLimitNs.
+__device__ bool wait_flag(const unsigned long long* f, unsigned long long want, const volatile int* abort) {
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(f) : "memory");
+    if (v == want) return true;
+    if (*abort) return false;
+    if (globaltimer() - t0 > kWaitLimitNs) return false;
+    __nanosleep(64);
+  }
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ Params p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -412,6 +438,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&sm.sum_bar), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.pub_bar), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.last_bar), 1);
+    mbar_init(smem_u32(&sm.mrg_full), 1);
     sm.abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&p.tm_ckv);
@@ -665,7 +692,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int b, begin, end, len, base;
     bool whole;
     uint32_t tb = 0;           // global tile counter
-    uint32_t nseg = 0, npart = 0;
+    uint32_t nseg = 0, npart = 0, npub = 0, nmrg = 0;
     bool ok = true;
     bool first_seg = true;     // the first segment of the range uses partial slot 2c, the last 2c + 1
     auto wait_or_fail = [&](uint32_t bar, uint32_t par, bool cl_scope) {
@@ -861,75 +888,166 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (rank == 0 && half == 0 && p.lse != nullptr)
           p.lse[(int64_t)b * kNH + h] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
       } else {
-        // ---- partial: publish (O, m, l) in this segment's slot; the last of the sequence's
-        // clusters to arrive (per latent half) merges every partial into ctx
+        // ---- partial: the last of the sequence's clusters to arrive (per latent half) merges every
+        // partial into ctx; the others publish (O, m, l) in their segment's slot and then raise the
+        // slot's ready flag.  Counting the arrival first means the merger never writes its own
+        // partial, and every cluster it then waits for has already arrived (so it is running) and
+        // needs nothing from the merger, so the wait ends.
         const int own = 2 * cl + (first_seg ? 0 : 1);
-        float* out = p.ws_o + (((int64_t)own * 2 + rank) * 256 + 128 * half) * kNH + h;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-          uint32_t r[32];
-          tmem_ld32(tO + c * 32, r);
-          tmem_ld_wait();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) out[(c * 32 + k) * kNH] = __uint_as_float(r[k]);
-        }
-        if (half == 0) p.ws_ml[((int64_t)own * 2 + rank) * kNH + h] = make_float2(m_run, l_tot);
-        __threadfence();
-        warp_arrive(smem_u32(&sm.pub_bar));
         if (sw == 0 && lane == 0) {
-          bool last = false;
-          if (mbar_wait(smem_u32(&sm.pub_bar), npart & 1u, abort_flag, kWaitLimitNs)) {
-            const int ns = list_slots(p, sm, base, tiles_of(len));
-            __threadfence();
-            last = arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err);
-            if (last) __threadfence();
-          } else {
-            fail_timeout(sm, p.err);
-          }
-          sm.is_last = last ? 1 : 0;
+          const int ns = list_slots(p, sm, base, tiles_of(len));
+          sm.is_last = arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0;
           mbar_arrive(smem_u32(&sm.last_bar));
         }
         if (!wait_or_fail(smem_u32(&sm.last_bar), npart & 1u, false)) break;
         ++npart;
-        if (sm.is_last) {
+        // A partial is this segment's context normalised by its own softmax sum, in bf16: head-major
+        // rows of 256 features (512 B) whose 16-byte chunks are rotated by (head & 15), so that eight
+        // consecutive heads reading the same chunk hit eight distinct bank groups.  This warp holds
+        // features [128 half, 128 half + 128) = chunks [16 half, 16 half + 16) of its head's row.
+        const float inv_own = 1.f / l_tot;
+        const int cswz = h & 15;
+        if (!sm.is_last) {
+          uint4* row = reinterpret_cast<uint4*>(p.ws_o) + (((int64_t)own * 2 + rank) * kNH + h) * 32;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tO + c * 32, r);
+            tmem_ld_wait();
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int chunk = 16 * half + 4 * c + v;
+              row[chunk ^ cswz] = make_uint4(
+                  pack_bf16x2(__uint_as_float(r[8 * v]) * inv_own, __uint_as_float(r[8 * v + 1]) * inv_own),
+                  pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_own, __uint_as_float(r[8 * v + 3]) * inv_own),
+                  pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_own, __uint_as_float(r[8 * v + 5]) * inv_own),
+                  pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_own, __uint_as_float(r[8 * v + 7]) * inv_own));
+            }
+          }
+          if (half == 0) p.ws_ml[((int64_t)own * 2 + rank) * kNH + h] = make_float2(m_run, l_tot);
           __threadfence();
-          // the other partials come from other SMs: read them through L2 (ld.global.cg).  Every
-          // sum runs in slot order with this CTA's own partial (kept in TMEM) in its slot's place,
-          // so the result does not depend on which cluster arrived last.
+          warp_arrive(smem_u32(&sm.pub_bar));
+          if (sw == 0 && lane == 0) {
+            if (mbar_wait(smem_u32(&sm.pub_bar), npub & 1u, abort_flag, kWaitLimitNs)) {
+              __threadfence();
+              st_release_gpu(p.ws_ready + 2 * (int64_t)own + rank, p.epoch);
+            } else {
+              fail_timeout(sm, p.err);
+            }
+          }
+          ++npub;
+        } else {
           const int ns = sm.nslots;
-          auto ml_of = [&](int sl) {
-            return sl == own ? make_float2(m_run, l_tot) : __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
-          };
-          float M = -INFINITY;
-          for (int i = 0; i < ns; ++i) M = fmaxf(M, ml_of(sm.slots[i]).x);
-          float L = 0.f;
-          for (int i = 0; i < ns; ++i) {
-            const float2 ml = ml_of(sm.slots[i]);
-            L += ml.y * ex2(ml.x - M);
+          // every other slot's partial has been published (lane 0 of each warp polls the flags)
+          int okw = 1;
+          if (lane == 0) {
+            for (int i = 0; i < ns && okw; ++i)
+              if (sm.slots[i] != own)
+                okw = wait_flag(p.ws_ready + 2 * (int64_t)sm.slots[i] + rank, p.epoch, abort_flag) ? 1 : 0;
+            if (!okw) fail_timeout(sm, p.err);
+          }
+          if (!__shfl_sync(0xffffffffu, okw, 0)) {
+            ok = false;
+            break;
+          }
+          // One other partial, and no further cache tiles will land in the stage buffers (this is the
+          // range's last segment and all its P*V products are complete): bulk-load the other
+          // partial (64 KB) into the stages.  Otherwise read the partials through L2.
+          int other = -1;
+          for (int i = 0; i < ns; ++i)
+            if (sm.slots[i] != own) other = sm.slots[i];
+          const bool bulk = (ns == 2) && (base + end >= sm.hi);
+          if (bulk) {
+            if (sw == 0 && lane == 0) {
+              fence_proxy_async_global();  // the partial was written through the generic proxy
+              const uint32_t bar = smem_u32(&sm.mrg_full);
+              mbar_arrive_expect_tx(bar, kNH * 512 + kNH * 8);
+              const uint8_t* src = reinterpret_cast<const uint8_t*>(p.ws_o) + ((int64_t)other * 2 + rank) * kNH * 512;
+#pragma unroll
+              for (int q = 0; q < 2; ++q) bulk_load_g2s(smem_u32(stages) + q * 32768, src + q * 32768, 32768, bar);
+              // and its (m, l) pairs, right after the partial
+              bulk_load_g2s(smem_u32(stages) + kNH * 512, p.ws_ml + ((int64_t)other * 2 + rank) * kNH, kNH * 8, bar);
+            }
+            if (!wait_or_fail(smem_u32(&sm.mrg_full), nmrg & 1u, false)) break;
+            ++nmrg;
+          }
+          // Weights of the slots (the softmax sums rescaled to the common maximum), then the sum over
+          // the slots in slot order, this CTA's own partial rounded to bf16 like the others: the
+          // result does not depend on which cluster arrived last.
+          float M, L, w_own = 0.f, w_other = 0.f;
+          if (bulk) {
+            const float2 ml = reinterpret_cast<const float2*>(stages + kNH * 512)[h];
+            M = fmaxf(m_run, ml.x);
+            // the same sum in either arrival order: two rounded terms, added once
+            const float a = l_tot * ex2(m_run - M), c = ml.y * ex2(ml.x - M);
+            L = a + c;
+            w_own = a / L;
+            w_other = c / L;
+          } else {
+            M = -INFINITY;
+            for (int i = 0; i < ns; ++i) {
+              const int sl = sm.slots[i];
+              M = fmaxf(M, sl == own ? m_run : __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h).x);
+            }
+            L = 0.f;
+            for (int i = 0; i < ns; ++i) {
+              const int sl = sm.slots[i];
+              const float2 ml = sl == own ? make_float2(m_run, l_tot) : __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
+              L += ml.y * ex2(ml.x - M);
+            }
           }
           const float inv = 1.f / L;
+          const uint4* srow = reinterpret_cast<const uint4*>(stages) + h * 32;
           __nv_bfloat16* dst = p.ctx + ((int64_t)b * kNH + h) * kDC + 256 * rank + 128 * half;
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t r[32];
             tmem_ld32(tO + c * 32, r);
             tmem_ld_wait();
+            float own_v[32];  // own partial, normalised and rounded through bf16 like a published one
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const uint32_t pr = pack_bf16x2(__uint_as_float(r[2 * k]) * inv_own, __uint_as_float(r[2 * k + 1]) * inv_own);
+              own_v[2 * k] = bf16_lo(pr);
+              own_v[2 * k + 1] = bf16_hi(pr);
+            }
             float acc[32];
+            if (bulk) {
+              // two slots: a sum of two rounded products is the same in either order
 #pragma unroll
-            for (int k = 0; k < 32; ++k) acc[k] = 0.f;
-            for (int i = 0; i < ns; ++i) {
-              const int sl = sm.slots[i];
-              const float w = ex2(ml_of(sl).x - M) * inv;
-              if (sl == own) {
+              for (int v = 0; v < 4; ++v) {
+                const uint4 u = srow[(16 * half + 4 * c + v) ^ cswz];
+                const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-                for (int k = 0; k < 32; ++k) acc[k] = fmaf(w, __uint_as_float(r[k]), acc[k]);
-              } else {
-                const float* src = p.ws_o + (((int64_t)sl * 2 + rank) * 256 + 128 * half + c * 32) * kNH + h;
-                float o[32];
+                for (int q = 0; q < 4; ++q) {
+                  acc[8 * v + 2 * q] = w_own * own_v[8 * v + 2 * q] + w_other * bf16_lo(uw[q]);
+                  acc[8 * v + 2 * q + 1] = w_own * own_v[8 * v + 2 * q + 1] + w_other * bf16_hi(uw[q]);
+                }
+              }
+            } else {
 #pragma unroll
-                for (int k = 0; k < 32; ++k) o[k] = __ldcg(src + k * kNH);
+              for (int k = 0; k < 32; ++k) acc[k] = 0.f;
+              for (int i = 0; i < ns; ++i) {
+                const int sl = sm.slots[i];
+                if (sl == own) {
+                  const float w = l_tot * ex2(m_run - M) * inv;
 #pragma unroll
-                for (int k = 0; k < 32; ++k) acc[k] = fmaf(w, o[k], acc[k]);
+                  for (int k = 0; k < 32; ++k) acc[k] = fmaf(w, own_v[k], acc[k]);
+                } else {
+                  const float2 ml = __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
+                  const float w = ml.y * ex2(ml.x - M) * inv;
+                  const uint4* grow = reinterpret_cast<const uint4*>(p.ws_o) + (((int64_t)sl * 2 + rank) * kNH + h) * 32;
+#pragma unroll
+                  for (int v = 0; v < 4; ++v) {
+                    const uint4 u = __ldcg(grow + ((16 * half + 4 * c + v) ^ cswz));
+                    const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                      acc[8 * v + 2 * q] = fmaf(w, bf16_lo(uw[q]), acc[8 * v + 2 * q]);
+                      acc[8 * v + 2 * q + 1] = fmaf(w, bf16_hi(uw[q]), acc[8 * v + 2 * q + 1]);
+                    }
+                  }
+                }
               }
             }
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
@@ -940,6 +1058,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           if (rank == 0 && half == 0 && p.lse != nullptr)
             p.lse[(int64_t)b * kNH + h] = (M + log2f(L)) * 0.69314718055994531f;
+          // the flags go back to zero for the next launch (which may reuse this launch's epoch when
+          // it replays a captured graph)
+          if (sw == 0 && lane == 0)
+            for (int i = 0; i < ns; ++i)
+              if (sm.slots[i] != own) p.ws_ready[2 * (int64_t)sm.slots[i] + rank] = 0ull;
         }
       }
       first_seg = false;
@@ -970,9 +1093,12 @@ size_t smem_bytes() { return (size_t)kSmemOff + sizeof(Smem) + 1024; }
 static_assert(kSmemOff + sizeof(Smem) + 1024 <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
 
 // Workspace layout for n_clusters clusters and B sequences: partial O, partial (m, l), counters.
-size_t ws_o_bytes(size_t nc) { return 2 * nc * 2 * 128 * 256 * sizeof(float); }
+size_t ws_o_bytes(size_t nc) { return 2 * nc * 2 * 128 * 256 * sizeof(__nv_bfloat16); }
 size_t ws_ml_bytes(size_t nc) { return 2 * nc * 2 * 128 * sizeof(float2); }
-size_t ws_bytes(size_t nc, size_t B) { return ws_o_bytes(nc) + ws_ml_bytes(nc) + B * 2 * sizeof(unsigned long long) + 256; }
+size_t ws_ready_bytes(size_t nc) { return 2 * nc * 2 * sizeof(unsigned long long); }
+size_t ws_bytes(size_t nc, size_t B) {
+  return ws_o_bytes(nc) + ws_ml_bytes(nc) + ws_ready_bytes(nc) + B * 2 * sizeof(unsigned long long) + 256;
+}
 
 // A launch identifier for the arrival counters: unique within the process (a 56-bit counter
 // started from the clock), never 0.
@@ -1057,6 +1183,8 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   w += ws_o_bytes(nc);
   p.ws_ml = reinterpret_cast<float2*>(w);
   w += ws_ml_bytes(nc);
+  p.ws_ready = reinterpret_cast<unsigned long long*>(w);
+  w += ws_ready_bytes(nc);
   p.ws_ctr = reinterpret_cast<unsigned long long*>(w);
   p.epoch = next_epoch();
   p.err = a.err;
@@ -1077,13 +1205,14 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
 // only holds pointers handed to it by someone else.  For them the split-KV scratch lives in this
 // file-scope array, which every GPU that loads the library holds until the process exits.
 // Sized for 74 clusters (one CTA pair per two SMs of a 148-SM B200) and up to 4096 sequences:
-// 74 x 2 partial slots of 128 heads x 512 fp32 features, their (m, l) pairs and two arrival
-// counters per sequence, about 37.2 MiB.
+// 74 x 2 partial slots of 128 heads x 512 bf16 features, their (m, l) pairs and ready flags, and
+// two arrival counters per sequence, about 18.9 MiB.
 namespace {
 constexpr size_t kStaticMaxClusters = 74;
 constexpr size_t kStaticMaxBatch = 4096;
-constexpr size_t kStaticScratchBytes = 2 * kStaticMaxClusters * 2 * 128 * 256 * sizeof(float) +
+constexpr size_t kStaticScratchBytes = 2 * kStaticMaxClusters * 2 * 128 * 256 * sizeof(__nv_bfloat16) +
                                        2 * kStaticMaxClusters * 2 * 128 * sizeof(float2) +
+                                       2 * kStaticMaxClusters * 2 * sizeof(unsigned long long) +
                                        kStaticMaxBatch * 2 * sizeof(unsigned long long) + 256;
 static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 }  // namespace

@@ -136,15 +136,16 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
  *   For callers that cannot allocate device memory around a decode call: a plugin / engine host
  *   whose enqueue path may not call cudaMalloc, code issuing work while a stream is being captured
  *   into a CUDA graph, or a caller that only holds pointers handed to it.  The split-KV scratch is
- *   a file-scope device array of 38,950,184 bytes (about 37.1 MiB: 74 clusters x 2 partial slots),
- *   held by every GPU that loads the library until the process exits.
+ *   a file-scope device array of 19,769,920 bytes (about 18.9 MiB: 74 clusters x 2 bf16 partial
+ *   slots), held by every GPU that loads the library until the process exits.
  *   Arguments and results are those of mla_decode_absorb with topk_idx = NULL and without
  *   workspace / ws_bytes.  dtype must be MLA_BF16 (else MLA_ERR_UNSUPPORTED); a device that would
  *   need more scratch than the array holds (more than 148 SMs) gets MLA_ERR_WORKSPACE.
  *   The first call on a device looks up the array's device address (cudaGetSymbolAddress, with
  *   that device current) and caches it; make that first call before any stream capture begins.
  *   Every call shares the one array and it keeps the last call's contents; nothing in it needs to
- *   start at zero (each byte a call reads was written earlier in the same call), but calls whose
+ *   start at zero (each byte a call reads was written earlier in the same call, and its arrival
+ *   counters and partial-ready flags carry a per-launch tag), but calls whose
  *   work overlaps on the GPU (different streams, or different host threads) race on it: serialise
  *   them.  No allocation of any kind happens inside this call.  Asynchronous on `stream`.
  */
