@@ -112,6 +112,7 @@ struct Smem {
   int abort;
   int lo, hi, b0, t_b0;  // tile range [lo, hi) in the global tile order, its first sequence and
                          // that sequence's first global tile
+  int len0;              // length of sequence b0 (clamped), so the first segment needs no reload
   int chunk;             // > 0: chunked plan, every cluster holds <= chunk tiles of one sequence
   int item0, kb;         // chunked plan: first chunk of this cluster's sequence, its chunk count
   long long total;       // tiles of all sequences
@@ -174,14 +175,25 @@ struct PlanTiles {
   }
 };
 
+// ceil(a / c) for 0 <= a, 1 <= c < 2^22, from a float reciprocal of c with one integer correction
+// (the float quotient is within one of the exact one at these sizes).
+__device__ __forceinline__ int ceil_div_rc(int a, int c, float rc) {
+  const int n = a + c - 1;
+  int q = __float2int_rz((float)n * rc);
+  if (q * c > n) --q;
+  else if ((q + 1) * c <= n) ++q;
+  return q;
+}
+
 // Chunks of the chunked plan with chunk size c: the sum over sequences of ceil(tiles / c).
 __device__ int chunk_items(const Params& p, const PlanTiles& pt, int c, int lane) {
   int n = 0;
   const int nk = (p.B + 31) / 32;
+  const float rc = 1.f / (float)c;
 #pragma unroll
   for (int k = 0; k < kPlanRegs; ++k)
-    if (k < nk) n += (pt.t[k] + c - 1) / c;
-  for (int k = kPlanRegs; k < nk; ++k) n += (pt.at(p, k, lane) + c - 1) / c;
+    if (k < nk) n += ceil_div_rc(pt.t[k], c, rc);
+  for (int k = kPlanRegs; k < nk; ++k) n += ceil_div_rc(pt.at(p, k, lane), c, rc);
   return warp_sum_i(n);
 }
 
@@ -191,7 +203,7 @@ __device__ int chunk_items(const Params& p, const PlanTiles& pt, int c, int lane
 __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
   PlanTiles pt;
   long long total = 0;
-  int maxt = 0, nonempty = 0;
+  int maxt = 0, mint = 1 << 30, nonempty = 0;
   bool bad = false;
   const int nk = (p.B + 31) / 32;
   for (int k = 0; k < nk; ++k) {
@@ -206,6 +218,7 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
     for (int i = 0; i < kPlanRegs; ++i)
       if (i == k) pt.t[i] = t;
     maxt = max(maxt, t);
+    if (t > 0) mint = min(mint, t);
     nonempty += t > 0 ? 1 : 0;
     total += t;
   }
@@ -213,6 +226,7 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
   for (int i = 0; i < kPlanRegs; ++i)
     if (i >= nk) pt.t[i] = 0;
   maxt = warp_max_i(maxt);
+  mint = -warp_max_i(-mint);
   nonempty = warp_sum_i(nonempty);
   {
     long long v = total;
@@ -228,6 +242,12 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
   if (nonempty > 0 && nonempty <= nc) {
     // chunk_items(maxt) = nonempty <= nc; below the balanced share it exceeds nc
     int lo = max(1, min(balanced, maxt)), hi = maxt;
+    if (mint == maxt) {
+      // every non-empty sequence has T = maxt tiles: at most q = nc / nonempty chunks each, so the
+      // smallest fitting chunk is ceil(T / q)
+      const int q = (int)(nc / nonempty);
+      lo = hi = (maxt + q - 1) / q;
+    }
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
       if (chunk_items(p, pt, mid, lane) <= nc) hi = mid;
@@ -292,11 +312,14 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
       base += __shfl_sync(0xffffffffu, inc, 31);
     }
   }
+  // length of the first sequence, read once here so the first segment needs no reload
+  const int len0 = (first_b < p.B) ? clamp_len(p.lengths[first_b], p.n_max) : 0;
   if (lane == 0) {
     sm.lo = lo;
     sm.hi = hi;
     sm.b0 = first_b;
     sm.t_b0 = t_first;
+    sm.len0 = len0;
     sm.chunk = chunk;
     sm.item0 = item0;
     sm.kb = kb;
@@ -307,16 +330,19 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
 
 // Walks the segments (sequence, first tile, end tile) of this cluster's range.
 struct SegIter {
-  int b, tb, t, hi;
+  int b, tb, t, hi, len0;
+  bool first;
   const int32_t* lengths;
   int n_max, B;
-  __device__ SegIter(const Smem& sm, const Params& p) : b(sm.b0), tb(sm.t_b0), t(sm.lo), hi(sm.hi),
-                                                        lengths(p.lengths), n_max(p.n_max), B(p.B) {}
+  __device__ SegIter(const Smem& sm, const Params& p)
+      : b(sm.b0), tb(sm.t_b0), t(sm.lo), hi(sm.hi), len0(sm.len0), first(true), lengths(p.lengths),
+        n_max(p.n_max), B(p.B) {}
   // On success: sequence b, tiles [begin, end) of it, its length, whether the range holds all of it,
   // and the global index of its first tile.
   __device__ bool next(int& sb, int& begin, int& end, int& len, bool& whole, int& base) {
     while (t < hi && b < B) {
-      len = clamp_len(lengths[b], n_max);
+      len = first ? len0 : clamp_len(lengths[b], n_max);
+      first = false;
       const int nt = tiles_of(len);
       if (tb + nt <= t) {  // sequence entirely before t (or empty)
         tb += nt;
@@ -454,7 +480,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync();  // the peer's barriers are initialised before any remote arrive
+  // The peer's barriers must be initialised before any remote arrive or copy: every warp arrives on
+  // the cluster barrier now and waits before its first remote operation.  The producer only touches
+  // this CTA's memory, so it starts loading before it waits.
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+  if (warp != 0) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   const uint32_t tmem = sm.tmem_base;
 
   if (warp == 0) {
@@ -500,6 +530,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_wait(smem_u32(&sm.full[k % kStages]), (k / kStages) & 1u, abort_flag, kWaitLimitNs);
       if (q_issued) mbar_wait(smem_u32(&sm.q_tma), 0, abort_flag, kWaitLimitNs);
     }
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     // lengths outside [1, n_max] (an error already flagged): sequences left without tiles get a
     // zero context and lse = -inf from cluster 0, each CTA its latent half
     if (cl == 0 && sm.bad) {
