@@ -62,4 +62,23 @@ struct PrefillArgs {
   void* kv;  // expanded [B, S, n_h, d_h + d_v] in the input dtype
 };
 
+// Launch with programmatic stream serialization: the kernel may start while the preceding kernel
+// in the stream is still running, and synchronises with it through griddepcontrol.wait before it
+// touches that kernel's data (every kernel of this library does).
+template <typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(Args...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 }  // namespace mla

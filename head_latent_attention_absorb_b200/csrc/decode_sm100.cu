@@ -439,6 +439,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const uint32_t rank = cluster_ctarank(), peer = rank ^ 1u;
   const int cl = blockIdx.x >> 1;
 
+  // The next kernel (the up-projection) may start its weight loads on SMs this grid leaves free.
+  // This kernel's own set-up and plan need nothing from the preceding kernel (the absorbed query);
+  // the threads that read its output or write memory it may read wait for it first (griddep_wait).
+  griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(smem_u32(&sm.full[s]), 1);
@@ -498,6 +502,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool ok = true, q_issued = false;
       while (ok && seg.next(b, begin, end, len, whole, base)) {
         if (!q_issued) {
+          griddep_wait();  // the absorbed query is the preceding kernel's output
           // the first sequence's query (this CTA's halves) goes in ahead of the cache tiles: latent
           // half into the four exchange buffers (free until the first exchange), rotary half apart
           const uint32_t qb = smem_u32(&sm.q_tma);
@@ -532,6 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
     __syncwarp();
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    griddep_wait();
     // lengths outside [1, n_max] (an error already flagged): sequences left without tiles get a
     // zero context and lse = -inf from cluster 0, each CTA its latent half
     if (cl == 0 && sm.bad) {
@@ -703,6 +709,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps (kBWarp0..)
+    griddep_wait();  // they read the absorbed query and write the context / workspace
     const int sw = warp - kBWarp0;
     const int half = sw >> 2;                        // which 32 keys of each tile
     const int quad = warp & 3;                       // TMEM lane quadrant of this warp
@@ -1224,8 +1231,7 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   const size_t smem = smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  decode_kernel<<<2 * nc, kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(decode_kernel, dim3(2 * nc), dim3(kThreads), smem, st, p);
 }
 
 // ------------------------------------------------------------------------------------------

@@ -65,6 +65,7 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
   const uint32_t ncols = tmem_cols_for(n);
   const uint32_t b_chunk_bytes = (uint32_t)n * 128;
 
+  griddep_launch_dependents();  // the next kernel may run its independent prologue
   if (threadIdx.x == 0) {
     for (int j = 0; j < S::kChunks; ++j) mbar_init(smem_u32(&full[j]), 1);
     mbar_init(smem_u32(&done), 1);
@@ -85,6 +86,7 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
   if (threadIdx.x == 0) {
     // ---- loads: K chunk j = features [64 j, 64 j + 64) of the contraction
     const uint64_t pol_w = policy_evict_first(), pol_a = policy_evict_last();
+    // the weights are no kernel's output: load them before waiting for the preceding kernel
     for (int j = 0; j < S::kChunks; ++j) {
       const uint32_t bar = smem_u32(&full[j]);
       mbar_arrive_expect_tx(bar, S::kAChunkBytes + b_chunk_bytes);
@@ -98,8 +100,11 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
         // W^UV_h rows d in [0, 128), latent columns [64 j, 64 j + 64): K-major A
         tma_load_2d(a_dst, &p.tm_w, bar, 64 * j, h * kRowsPerHead + kDH, pol_w);
       }
-      tma_load_3d(smem_u32(b_s + j * b_chunk_bytes), &p.tm_act, bar, 64 * j, h, b0, pol_a);
     }
+    // the activations (and the output this kernel overwrites) belong to the preceding kernels
+    griddep_wait();
+    for (int j = 0; j < S::kChunks; ++j)
+      tma_load_3d(smem_u32(b_s + j * b_chunk_bytes), &p.tm_act, smem_u32(&full[j]), 64 * j, h, b0, pol_a);
     // ---- MMAs: D[128 x n] (+)= A_j B_j^T over the chunks as they land
     const uint32_t idesc = idesc_bf16_f32(128, (uint32_t)n, kAbsorb ? 1u : 0u, 0u);
     bool ok = true;
@@ -125,6 +130,7 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
   __syncwarp();
 
   // ---- epilogue: lane i of warp w holds row 32 w + i of D (a latent feature / value feature)
+  griddep_wait();  // every thread that writes the output waits for the preceding kernel
   const bool ok = mbar_wait(smem_u32(&done), 0, &abort_flag, kWaitLimitNs);
   if (__all_sync(0xffffffffu, ok)) {
     tc_fence_after();
@@ -187,8 +193,7 @@ cudaError_t launch(int B, const void* act, int64_t ld_head, const void* w, void*
   cudaError_t e = cudaFuncSetAttribute(proj_kernel<kAbsorb>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(kAbsorb ? kDC / 128 : 1, kNH, (B + n_tile - 1) / n_tile);
-  proj_kernel<kAbsorb><<<grid, 128, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(proj_kernel<kAbsorb>, grid, dim3(128), smem, st, p);
 }
 
 }  // namespace proj_tc

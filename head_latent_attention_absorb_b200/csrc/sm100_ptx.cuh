@@ -98,6 +98,16 @@ __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
+// Programmatic dependent launch.  launch_dependents lets the next kernel in the stream (launched
+// with programmatic stream serialization) start its independent prologue once every CTA of this
+// grid has executed it; griddep_wait blocks the calling thread until the preceding grid has
+// completed and its memory operations are visible.  Both are no-ops for a kernel launched without
+// a programmatic predecessor / dependent.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Packed half-precision add (round to nearest).
 __device__ __forceinline__ uint32_t hadd2_u32(uint32_t a, uint32_t b) {
   uint32_t r;
