@@ -154,6 +154,68 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
+def time_secondary(dev, reps: int):
+    """The other workloads of the hot path, each timed on its own with CUDA events (L2 flushed
+    before every launch): the ragged long-context decode, the V3.2 top-k decode and the naive causal
+    prefill.  Reported beside the headline line; algorithmic bytes / FLOPs as for the headline."""
+    from head_latent_attention_absorb_b200 import api
+    from head_latent_attention_absorb_b200.configs import PREFILL, RAGGED_LONG, SPARSE_V32
+    from head_latent_attention_absorb_b200.inputs import make_prefill_inputs
+    peaks = load_peaks()
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn):
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps + 3)]
+        for e0, e1 in ev:
+            flush.zero_()
+            e0.record(stream); fn(); e1.record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev[3:])
+
+    out = {}
+    for cfg in (RAGGED_LONG, SPARSE_V32):
+        x = make_decode_inputs(cfg)
+        cache = x["cache"].to(dev)
+        c_kv, k_r = cache[..., :cfg.d_c], cache[..., cfg.d_c:]
+        w = x["w_kv_b"].to(dev)
+        qt = api.mla_absorb_q(cfg.dims, x["q_nope"].to(dev), w)
+        q_pe, lengths = x["q_pe"].to(dev), x["lengths"].to(dev)
+        topk = None if x["topk"] is None else x["topk"].to(dev)
+        ctx = torch.empty_like(qt)
+        ws = torch.empty((api.mla_decode_workspace_size(cfg.dims, torch.bfloat16, cfg.B, cfg.n_max,
+                                                        0 if topk is None else cfg.topk),), dtype=torch.uint8,
+                         device=dev)
+        ms = timed(lambda: api.mla_decode_absorb(cfg.dims, qt, q_pe, c_kv, k_r, lengths, cfg.scale, topk_idx=topk,
+                                                 ctx=ctx, workspace=ws, stream=stream))
+        keys = cfg.B * cfg.topk if topk is not None else int(x["lengths"].sum())
+        nbytes = keys * (cfg.d_c + cfg.d_r) * 2 + cfg.B * cfg.n_h * (2 * cfg.d_c + cfg.d_r) * 2
+        if topk is not None:
+            nbytes += cfg.B * cfg.topk * 4
+        flops = 2 * keys * cfg.n_h * (2 * cfg.d_c + cfg.d_r)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out[cfg.name] = {"call": "mla_decode_absorb", "ms": ms, "tokens_per_s": cfg.B / (ms * 1e-3),
+                         "keys": keys, "algorithmic_bytes": nbytes, "achieved_GBs": gbs,
+                         "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": flops / (ms * 1e-3) / 1e12}
+        del x, cache, c_kv, k_r, ws
+        torch.cuda.empty_cache()
+    cfg = PREFILL
+    p = make_prefill_inputs(cfg)
+    q, c_kv, k_r, w = p["q"].to(dev), p["c_kv"].to(dev), p["k_r"].to(dev), p["w_kv_b"].to(dev)
+    o = torch.empty((cfg.B, cfg.n_max, cfg.n_h, cfg.d_v), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty((api.mla_prefill_workspace_size(cfg.dims, torch.bfloat16, cfg.B, cfg.n_max),),
+                     dtype=torch.uint8, device=dev)
+    ms = timed(lambda: api.mla_prefill_naive(cfg.dims, q, c_kv, k_r, w, cfg.scale, out=o, workspace=ws,
+                                             stream=stream))
+    S, B = cfg.n_max, cfg.B
+    flops = 2 * B * S * cfg.n_h * (cfg.d_h + cfg.d_v) * cfg.d_c \
+        + 2 * B * cfg.n_h * (S * (S + 1) // 2) * ((cfg.d_h + cfg.d_r) + cfg.d_v)
+    tf = flops / (ms * 1e-3) / 1e12
+    out[cfg.name] = {"call": "mla_prefill_naive", "ms": ms, "tokens_per_s": B * S / (ms * 1e-3), "flops": flops,
+                     "tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"]}
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     from head_latent_attention_absorb_b200 import api
     dev = torch.device("cuda", local_rank)
@@ -299,6 +361,7 @@ def run_ours(args, rank, world, local_rank):
                 "note": "queries copied from pinned host memory and outputs read back every step; cache and "
                         "wkv_b resident"},
         "gpu_launches": n_launch * K,
+        "secondary": None if args.no_secondary else time_secondary(dev, 10),
         "clocks": clocks,
         "wall_s_timed_region": t_wall,
     }
@@ -313,6 +376,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the timings of the ragged, top-k and prefill workloads")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world = int(os.environ.get("WORLD_SIZE", "1"))

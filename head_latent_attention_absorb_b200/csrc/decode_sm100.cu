@@ -79,6 +79,11 @@ struct Params {
   CUtensorMap tm_kr;   // 3-D (d_r, n_max, B), box (32, 64, 1), 64-byte swizzle
   CUtensorMap tm_q;    // 2-D (d_c, B * 128) rows of q~, box (64, 128), 128-byte swizzle
   CUtensorMap tm_qp;   // 2-D (d_r, B * 128) rows of q^R, box (32, 128), 64-byte swizzle
+  const int32_t* topk_idx;  // [B][topk] positions attended (distinct), or null for the dense decode
+  int topk;
+  const __nv_bfloat16* c_kv_base;  // sparse: row r = sequence * n_max + position at c_kv_base + r * ckv_row
+  const __nv_bfloat16* k_r_base;
+  int64_t ckv_row, kr_row;
   const __nv_bfloat16* q_tilde;
   int64_t ldqt;
   const __nv_bfloat16* q_pe;
@@ -105,6 +110,7 @@ struct Smem {
   uint64_t red_bar[2][4], sum_bar; // row-max rendezvous of the two warps of a lane quadrant / final sum
   uint64_t pub_bar, last_bar;      // partial published by all softmax warps / merge decision made
   uint64_t mrg_full;               // the other cluster's partial bulk-loaded for the merge
+  uint64_t mrg_full2[2], mrg_empty2[2];  // streamed merge of several partials (double-buffered)
   float red[2][2][kNH];            // [tile parity][key half][head] partial row max
   float lsum[2][kNH];              // [key half][head] partial softmax sum
   int16_t slots[kMaxClusters];     // partial slots of the sequence being merged
@@ -156,7 +162,12 @@ __device__ __forceinline__ int cluster_of(long long t, long long total, long lon
   return (int)c;
 }
 
-__device__ __forceinline__ int seq_tiles(const Params& p, int b) { return tiles_of(clamp_len(p.lengths[b], p.n_max)); }
+// Keys a sequence attends: its cached length (dense), or the top-k set size (sparse: every sequence
+// attends exactly topk gathered positions, which must lie in [0, length)).
+__device__ __forceinline__ int seq_len(const Params& p, int b) {
+  return p.topk > 0 ? p.topk : clamp_len(p.lengths[b], p.n_max);
+}
+__device__ __forceinline__ int seq_tiles(const Params& p, int b) { return tiles_of(seq_len(p, b)); }
 
 // Tile counts of the first 256 sequences stay in registers (lane l holds sequences l + 32 k);
 // later ones are re-read from global memory.
@@ -212,7 +223,7 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
     if (b < p.B) {
       const int len = p.lengths[b];
       bad |= (len < 1 || len > p.n_max);
-      t = tiles_of(clamp_len(len, p.n_max));
+      t = tiles_of(p.topk > 0 ? p.topk : clamp_len(len, p.n_max));
     }
 #pragma unroll
     for (int i = 0; i < kPlanRegs; ++i)
@@ -296,7 +307,7 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
     int base = 0;  // tiles before batch b0
     for (int b0 = 0; b0 < p.B && first_b == p.B; b0 += 32) {
       const int b = b0 + lane;
-      const int t = b < p.B ? tiles_of(clamp_len(p.lengths[b], p.n_max)) : 0;
+      const int t = b < p.B ? seq_tiles(p, b) : 0;
       int inc = t;  // inclusive prefix within the warp
       for (int o = 1; o < 32; o <<= 1) {
         const int v = __shfl_up_sync(0xffffffffu, inc, o);
@@ -313,7 +324,7 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
     }
   }
   // length of the first sequence, read once here so the first segment needs no reload
-  const int len0 = (first_b < p.B) ? clamp_len(p.lengths[first_b], p.n_max) : 0;
+  const int len0 = (first_b < p.B) ? seq_len(p, first_b) : 0;
   if (lane == 0) {
     sm.lo = lo;
     sm.hi = hi;
@@ -333,15 +344,15 @@ struct SegIter {
   int b, tb, t, hi, len0;
   bool first;
   const int32_t* lengths;
-  int n_max, B;
+  int n_max, B, topk;
   __device__ SegIter(const Smem& sm, const Params& p)
       : b(sm.b0), tb(sm.t_b0), t(sm.lo), hi(sm.hi), len0(sm.len0), first(true), lengths(p.lengths),
-        n_max(p.n_max), B(p.B) {}
+        n_max(p.n_max), B(p.B), topk(p.topk) {}
   // On success: sequence b, tiles [begin, end) of it, its length, whether the range holds all of it,
   // and the global index of its first tile.
   __device__ bool next(int& sb, int& begin, int& end, int& len, bool& whole, int& base) {
     while (t < hi && b < B) {
-      len = first ? len0 : clamp_len(lengths[b], n_max);
+      len = first ? len0 : (topk > 0 ? topk : clamp_len(lengths[b], n_max));
       first = false;
       const int nt = tiles_of(len);
       if (tb + nt <= t) {  // sequence entirely before t (or empty)
@@ -445,7 +456,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(smem_u32(&sm.full[s]), 1);
+      // dense: the producer's arrive.expect_tx + the TMA bytes; sparse: one cp.async arrival per lane
+      mbar_init(smem_u32(&sm.full[s]), p.topk > 0 ? 32 : 1);
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     // softmax-side arrivals are one per softmax warp, after a __syncwarp
@@ -469,6 +481,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&sm.pub_bar), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.last_bar), 1);
     mbar_init(smem_u32(&sm.mrg_full), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&sm.mrg_full2[i]), 1);
+      mbar_init(smem_u32(&sm.mrg_empty2[i]), kSoftmaxWarps);
+    }
     sm.abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&p.tm_ckv);
@@ -493,7 +509,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // The whole warp walks the tiles (the control flow is the same in every lane).  Dense: lane 0
+    // issues one 3-D TMA box per 64-feature slab.  Sparse: the warp loads the tile's 64 selected
+    // positions (two per lane), checks them against the sequence length, and copies the rows with
+    // per-lane 16-byte cp.async into the layout the TMA boxes would give.
+    {
       const uint64_t pol = policy_evict_first();
       SegIter seg(sm, p);
       int b, begin, end, len, base;
@@ -505,35 +525,83 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           griddep_wait();  // the absorbed query is the preceding kernel's output
           // the first sequence's query (this CTA's halves) goes in ahead of the cache tiles: latent
           // half into the four exchange buffers (free until the first exchange), rotary half apart
-          const uint32_t qb = smem_u32(&sm.q_tma);
-          mbar_arrive_expect_tx(qb, kQLatBytes + kQRopeBytes);
+          if (lane == 0) {
+            const uint32_t qb = smem_u32(&sm.q_tma);
+            mbar_arrive_expect_tx(qb, kQLatBytes + kQRopeBytes);
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            tma_load_2d(smem_u32(xbuf + j * kXBytes), &p.tm_q, qb, 256 * (int)rank + 64 * j, b * kNH, pol);
-          tma_load_2d(smem_u32(qrope), &p.tm_qp, qb, 32 * (int)rank, b * kNH, pol);
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(smem_u32(xbuf + j * kXBytes), &p.tm_q, qb, 256 * (int)rank + 64 * j, b * kNH, pol);
+            tma_load_2d(smem_u32(qrope), &p.tm_qp, qb, 32 * (int)rank, b * kNH, pol);
+          }
           q_issued = true;
         }
+        const int seq_len_b = p.topk > 0 ? clamp_len(p.lengths[b], p.n_max) : 0;
         for (int i = begin; i < end && ok; ++i, ++it) {
           const uint32_t st = it % kStages, ph = (it / kStages) & 1u;
-          if (!mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
-            fail_timeout(sm, p.err);
+          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs))) {
+            if (lane == 0) fail_timeout(sm, p.err);
             ok = false;
             break;
           }
           const uint32_t dst = smem_u32(stages + st * kStageBytes);
           const uint32_t bar = smem_u32(&sm.full[st]);
-          mbar_arrive_expect_tx(bar, kStageBytes);
+          if (p.topk == 0) {
+            if (lane == 0) {
+              mbar_arrive_expect_tx(bar, kStageBytes);
 #pragma unroll
-          for (int s = 0; s < 4; ++s)
-            tma_load_3d(dst + s * kSlabBytes, &p.tm_ckv, bar, 256 * (int)rank + 64 * s, i * kTile, b, pol);
-          tma_load_3d(dst + kLatBytes, &p.tm_kr, bar, 32 * (int)rank, i * kTile, b, pol);
+              for (int s = 0; s < 4; ++s)
+                tma_load_3d(dst + s * kSlabBytes, &p.tm_ckv, bar, 256 * (int)rank + 64 * s, i * kTile, b, pol);
+              tma_load_3d(dst + kLatBytes, &p.tm_kr, bar, 32 * (int)rank, i * kTile, b, pol);
+            }
+          } else {
+            // rows of the 2-D caches: b * n_max + position; positions past the top-k set (the last
+            // tile's tail, zeroed before use) and invalid ones (flagged) read position 0
+            int rows[2];
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+              const int k = i * kTile + 32 * hf + lane;
+              int pos = 0;
+              if (k < p.topk) {
+                pos = p.topk_idx[(int64_t)b * p.topk + k];
+                if (pos < 0 || pos >= seq_len_b) {
+                  raise_error(p.err, MLA_ERR_INDEX);
+                  pos = 0;
+                }
+              }
+              rows[hf] = b * p.n_max + pos;
+            }
+            // Each lane copies 16-byte chunks (cp.async) straight into the swizzled layout a TMA box
+            // would produce: latent slab s, key k, chunk c at s * 8 KB + 128 k + 16 (c ^ (k & 7));
+            // rotary key k, chunk c at 32 KB + 64 k + 16 (c ^ ((k >> 1) & 3)).  Eight lanes cover one
+            // 128-byte row, so every instruction reads four whole rows and hits distinct banks.
+#pragma unroll 1
+            for (int g = 0; g < kTile / 4; ++g) {
+              const int key = 4 * g + (lane >> 3), ch = lane & 7;
+              const int r0 = __shfl_sync(0xffffffffu, rows[0], key & 31), r1 = __shfl_sync(0xffffffffu, rows[1], key & 31);
+              const __nv_bfloat16* src = p.c_kv_base + (int64_t)(key < 32 ? r0 : r1) * p.ckv_row + 256 * rank + 8 * ch;
+              const uint32_t d = dst + key * 128 + ((ch ^ (key & 7)) << 4);
+#pragma unroll
+              for (int s = 0; s < 4; ++s) cp_async_16(d + s * kSlabBytes, src + 64 * s);
+            }
+#pragma unroll 1
+            for (int g = 0; g < kTile / 8; ++g) {
+              const int key = 8 * g + (lane >> 2), ch = lane & 3;
+              const int r0 = __shfl_sync(0xffffffffu, rows[0], key & 31), r1 = __shfl_sync(0xffffffffu, rows[1], key & 31);
+              const __nv_bfloat16* src = p.k_r_base + (int64_t)(key < 32 ? r0 : r1) * p.kr_row + 32 * rank + 8 * ch;
+              cp_async_16(dst + kLatBytes + key * 64 + ((ch ^ ((key >> 1) & 3)) << 4), src);
+            }
+            cp_async_mbar_arrive(bar);  // this lane's copies of the tile, counted on full[st]
+          }
+          __syncwarp();
         }
       }
       // drain: every load issued must have landed before the CTA may exit
-      const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0;
-      for (uint32_t k = first; k < it; ++k)
-        mbar_wait(smem_u32(&sm.full[k % kStages]), (k / kStages) & 1u, abort_flag, kWaitLimitNs);
-      if (q_issued) mbar_wait(smem_u32(&sm.q_tma), 0, abort_flag, kWaitLimitNs);
+      if (lane == 0) {
+        const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0;
+        for (uint32_t k = first; k < it; ++k)
+          mbar_wait(smem_u32(&sm.full[k % kStages]), (k / kStages) & 1u, abort_flag, kWaitLimitNs);
+        if (q_issued) mbar_wait(smem_u32(&sm.q_tma), 0, abort_flag, kWaitLimitNs);
+      }
     }
     __syncwarp();
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -579,6 +647,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto issue_qk = [&](uint32_t t, int tile_in_seq) {
       const uint32_t st = t % kStages;
       if (!wait_or_fail(smem_u32(&sm.full[st]), (t / kStages) & 1u, false)) return;
+      if (p.topk > 0) fence_proxy_async_smem();  // rows copied by cp.async (generic proxy)
       const int valid = len - tile_in_seq * kTile;
       if (valid < kTile) {  // rows past the sequence end: zero them so 0 * garbage cannot occur
         uint8_t* sbase = stages + st * kStageBytes;
@@ -614,6 +683,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto issue_pv = [&](uint32_t t, bool first_of_seg) {
       if (!wait_or_fail(smem_u32(&sm.p_full), t & 1u, false)) return;
       tc_fence_after();
+      if (p.topk > 0) fence_proxy_async_smem();
       const uint32_t st = t % kStages;
       if (lane == 0) {
         const uint32_t base = smem_u32(stages + st * kStageBytes);
@@ -996,6 +1066,139 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int i = 0; i < ns; ++i)
             if (sm.slots[i] != own) other = sm.slots[i];
           const bool bulk = (ns == 2) && (base + end >= sm.hi);
+          if (ns > 2 && base + end >= sm.hi) {
+            // ---- several partials, and no further cache tiles will land in the stage buffers:
+            // stream the other partials through two 64 KB stage buffers (bulk loads, one ahead),
+            // accumulating in TMEM in slot order.  This CTA's own partial, normalised and rounded
+            // to bf16 like a published one, is kept in the TMEM columns the scores, P and the query
+            // used (free after the last tile); the O columns become the accumulator.
+            int own_pos = 0;
+            for (int i = 0; i < ns; ++i)
+              if (sm.slots[i] == own) own_pos = i;
+            const int n_other = ns - 1;
+            const bool issuer = (sw == 0 && lane == 0);
+            auto issue = [&](int k) {  // other partial k -> stage buffer k & 1
+              const int sl = sm.slots[k < own_pos ? k : k + 1];
+              const uint32_t buf = smem_u32(stages) + (k & 1) * 65536;
+              const uint32_t bar = smem_u32(&sm.mrg_full2[k & 1]);
+              mbar_arrive_expect_tx(bar, kNH * 512);
+              const uint8_t* src = reinterpret_cast<const uint8_t*>(p.ws_o) + ((int64_t)sl * 2 + rank) * kNH * 512;
+              bulk_load_g2s(buf, src, 32768, bar);
+              bulk_load_g2s(buf + 32768, src + 32768, 32768, bar);
+            };
+            if (issuer) {
+              fence_proxy_async_global();  // the partials were written through the generic proxy
+              issue(0);
+              if (n_other > 1) issue(1);
+            }
+            float M = m_run;
+#pragma unroll 4
+            for (int i = 0; i < ns; ++i)
+              if (sm.slots[i] != own) M = fmaxf(M, __ldcg(p.ws_ml + ((int64_t)sm.slots[i] * 2 + rank) * kNH + h).x);
+            float L = 0.f;
+#pragma unroll 4
+            for (int i = 0; i < ns; ++i) {
+              const int sl = sm.slots[i];
+              const float2 ml = sl == own ? make_float2(m_run, l_tot) : __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
+              L += ml.y * ex2(ml.x - M);
+            }
+            const float inv = 1.f / L;
+            const uint32_t tStash = tmem + lane_off + kColS + 64 * half;  // 64 columns of bf16 pairs
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t r[32], pr[16];
+              tmem_ld32(tO + c * 32, r);
+              tmem_ld_wait();
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                pr[k] = pack_bf16x2(__uint_as_float(r[2 * k]) * inv_own, __uint_as_float(r[2 * k + 1]) * inv_own);
+              tmem_st16(tStash + 16 * c, pr);
+            }
+            tmem_st_wait();
+            __nv_bfloat16* dst = p.ctx + ((int64_t)b * kNH + h) * kDC + 256 * rank + 128 * half;
+            int k = 0;
+            bool okm = true;
+            for (int i = 0; i < ns && okm; ++i) {
+              const int sl = sm.slots[i];
+              const bool mine = (sl == own);
+              float w;
+              const uint4* srow = nullptr;
+              if (mine) {
+                w = l_tot * ex2(m_run - M) * inv;
+              } else {
+                if (!wait_or_fail(smem_u32(&sm.mrg_full2[k & 1]), (k >> 1) & 1u, false)) {
+                  okm = false;
+                  break;
+                }
+                const float2 ml = __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
+                w = ml.y * ex2(ml.x - M) * inv;
+                srow = reinterpret_cast<const uint4*>(stages + (k & 1) * 65536) + h * 32;
+              }
+              const bool last_slot = (i + 1 == ns);
+#pragma unroll 1
+              for (int c = 0; c < 4; ++c) {
+                float acc[32];
+                if (i == 0) {
+#pragma unroll
+                  for (int q = 0; q < 32; ++q) acc[q] = 0.f;
+                } else {
+                  uint32_t r[32];
+                  tmem_ld32(tO + c * 32, r);
+                  tmem_ld_wait();
+#pragma unroll
+                  for (int q = 0; q < 32; ++q) acc[q] = __uint_as_float(r[q]);
+                }
+                uint32_t uw[16];
+                if (mine) {
+                  tmem_ld16(tStash + 16 * c, uw);
+                  tmem_ld_wait();
+                } else {
+#pragma unroll
+                  for (int v = 0; v < 4; ++v) {
+                    const uint4 u = srow[(16 * half + 4 * c + v) ^ cswz];
+                    uw[4 * v] = u.x; uw[4 * v + 1] = u.y; uw[4 * v + 2] = u.z; uw[4 * v + 3] = u.w;
+                  }
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                  acc[2 * q] = fmaf(w, bf16_lo(uw[q]), acc[2 * q]);
+                  acc[2 * q + 1] = fmaf(w, bf16_hi(uw[q]), acc[2 * q + 1]);
+                }
+                if (last_slot) {
+                  uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                  for (int v = 0; v < 4; ++v)
+                    d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                                       pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+                } else {
+                  uint32_t r[32];
+#pragma unroll
+                  for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(acc[q]);
+                  tmem_st32(tO + c * 32, r);
+                }
+              }
+              tmem_st_wait();
+              if (!mine) {
+                // this warp is done with stage buffer k & 1; once all are, it takes partial k + 2
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&sm.mrg_empty2[k & 1]));
+                if (issuer && k + 2 < n_other) {
+                  if (mbar_wait(smem_u32(&sm.mrg_empty2[k & 1]), (k >> 1) & 1u, abort_flag, kWaitLimitNs)) issue(k + 2);
+                  else fail_timeout(sm, p.err);
+                }
+                ++k;
+              }
+            }
+            if (!okm) {
+              ok = false;
+              break;
+            }
+            if (rank == 0 && half == 0 && p.lse != nullptr)
+              p.lse[(int64_t)b * kNH + h] = (M + log2f(L)) * 0.69314718055994531f;
+            if (sw == 0 && lane == 0)
+              for (int i = 0; i < ns; ++i)
+                if (sm.slots[i] != own) p.ws_ready[2 * (int64_t)sm.slots[i] + rank] = 0ull;
+          } else {
           if (bulk) {
             if (sw == 0 && lane == 0) {
               fence_proxy_async_global();  // the partial was written through the generic proxy
@@ -1102,6 +1305,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (sw == 0 && lane == 0)
             for (int i = 0; i < ns; ++i)
               if (sm.slots[i] != own) p.ws_ready[2 * (int64_t)sm.slots[i] + rank] = 0ull;
+          }
         }
       }
       first_seg = false;
@@ -1205,6 +1409,16 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
     if (!make_tensor_map_bf16(&p.tm_q, a.q_tilde, 2, qd, qs, qbox, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_tensor_map_bf16(&p.tm_qp, a.q_pe, 2, rd, rs, rbox, CU_TENSOR_MAP_SWIZZLE_64B))
       return cudaErrorInvalidValue;
+  }
+  if (a.topk > 0) {
+    // sparse: rows of the caches addressed as sequence * n_max + position (their batch stride is
+    // n_max rows; the caller checked)
+    p.topk_idx = a.topk_idx;
+    p.topk = a.topk;
+    p.c_kv_base = static_cast<const __nv_bfloat16*>(a.c_kv);
+    p.k_r_base = static_cast<const __nv_bfloat16*>(a.k_r);
+    p.ckv_row = a.ckv_r;
+    p.kr_row = a.kr_r;
   }
   p.q_tilde = static_cast<const __nv_bfloat16*>(a.q_tilde);
   p.ldqt = a.ldqt;

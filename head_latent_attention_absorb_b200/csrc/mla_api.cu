@@ -108,16 +108,22 @@ mla_status mla_absorb_q(mla_dims dims, mla_dtype dtype, int32_t B, const void* q
 
 size_t mla_decode_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
   if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
-  // bf16 dense decode runs the tensor-core kernel only; every other case the CUDA-core kernels
+  // bf16 runs the tensor-core kernel (the sparse variant falls back to the CUDA-core kernel for a
+  // cache whose batch stride is not n_max rows: size for both); fp32 the CUDA-core kernels
   if (dtype == MLA_BF16 && topk == 0) return mla::decode_tc_workspace(B);
   const int cap = topk > 0 ? topk : n_max;
-  return mla::decode_simt_workspace(dims.n_h, dims.d_c, B, cap);
+  const size_t simt = mla::decode_simt_workspace(dims.n_h, dims.d_c, B, cap);
+  if (dtype == MLA_BF16) {
+    const size_t tc = mla::decode_tc_workspace(B);
+    return tc > simt ? tc : simt;
+  }
+  return simt;
 }
 
 int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk) {
   if (check_dims(dims, dtype) != MLA_OK || B <= 0 || n_max <= 0 || topk < 0) return 0;
   const int cap = topk > 0 ? topk : n_max;
-  if (dtype == MLA_BF16 && topk == 0) return 1;  // tensor-core decode, partials merged in-kernel
+  if (dtype == MLA_BF16) return 1;  // tensor-core decode, partials merged in-kernel
   return mla::decode_simt_splits(B, cap) > 1 ? 2 : 1;
 }
 
@@ -165,7 +171,10 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B, const vo
   a.ctx = ctx_out; a.lse = lse_out; a.err = dev_err;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   cudaError_t e;
-  if (dtype == MLA_BF16 && !topk_idx)
+  // the sparse tensor-core path gathers rows of the caches viewed as 2-D (B * n_max rows)
+  const bool packed = (B == 1 || (ckv_bstride == (int64_t)n_max * ckv_rstride && kr_bstride == (int64_t)n_max * kr_rstride)) &&
+                      (int64_t)B * n_max < ((int64_t)1 << 31);
+  if (dtype == MLA_BF16 && (!topk_idx || packed))
     e = mla::decode_tc_launch(a, workspace, st);
   else if (dtype == MLA_BF16)
     e = mla::decode_simt_launch<__nv_bfloat16>(a, workspace, st);
