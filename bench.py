@@ -34,6 +34,17 @@ from head_latent_attention_absorb_b200.shard import max_over_ranks, shard_range 
 METRIC = "MLA absorbed-decode tokens/s and % of roofline (B=32, N=4096, 128 heads)"
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch on this workload,
+# from the ncu capture summarised in profiles/decode_kernel_v3_b32_n4096.md, valid only for the
+# kernel source it was taken on (sha256 prefix of csrc/decode_sm100.cu).
+DECODE_TRAFFIC = {"bytes": 155_826_176 + 3_898_368, "source_sha256": "42134f45759d00ea"}
+
+
+def decode_traffic():
+    import hashlib
+    src = os.path.join(ROOT, "head_latent_attention_absorb_b200", "csrc", "decode_sm100.cu")
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return DECODE_TRAFFIC["bytes"] if h == DECODE_TRAFFIC["source_sha256"] else None
 
 
 def load_peaks():
@@ -348,7 +359,7 @@ def run_ours(args, rank, world, local_rank):
                              "captured once), mean over steps, max over ranks; per-call times from separate "
                              "launches with events between the calls"},
         "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mla_decode_absorb",
+                     "frac": achieved_gbs / peaks["hbm_gbs"], "traffic": decode_traffic(), "kernel": "mla_decode_absorb",
                      "peak_source": peaks["source"] + " (hbm_gbs, burst)",
                      "algorithmic_bytes_per_launch": dec["bytes"], "ms_per_launch": ms_dec,
                      "tensor_achieved_tflops": achieved_tf, "tensor_peak_tflops": peaks["bf16_tflops"],
