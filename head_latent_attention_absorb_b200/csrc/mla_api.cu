@@ -257,8 +257,14 @@ mla_status mla_prefill_naive(mla_dims dims, mla_dtype dtype, int32_t B, int32_t 
   a.q = q; a.c_kv = c_kv; a.ckv_r = ckv_rstride; a.k_r = k_r; a.kr_r = kr_rstride; a.w = w_kv_b;
   a.scale = scale; a.out = out; a.kv = workspace;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  cudaError_t e = dtype == MLA_BF16 ? mla::prefill_simt_launch<__nv_bfloat16>(a, st)
-                                    : mla::prefill_simt_launch<float>(a, st);
+  cudaError_t e;
+  if (dtype == MLA_BF16) {
+    // tensor-core expansion (needs 16-byte-aligned rows for its TMA maps), then the attention
+    e = mla::expand_tc_launch(a, st);
+    if (e == cudaSuccess) e = mla::prefill_attn_simt_launch<__nv_bfloat16>(a, st);
+  } else {
+    e = mla::prefill_simt_launch<float>(a, st);
+  }
   return cuda_status(e, "mla_prefill_naive launch");
 }
 

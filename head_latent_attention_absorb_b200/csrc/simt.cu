@@ -348,6 +348,16 @@ cudaError_t decode_simt_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
 }
 
 template <typename T>
+cudaError_t prefill_attn_simt_launch(const PrefillArgs& a, cudaStream_t st) {
+  dim3 grid((a.n_h + 3) / 4, a.S, a.B);
+  if (a.d_h <= 32 && a.d_r <= 32 && a.d_v <= 32)
+    prefill_attn_simt<T, 1, 1, 1><<<grid, 128, 0, st>>>(a);
+  else
+    prefill_attn_simt<T, 8, 4, 8><<<grid, 128, 0, st>>>(a);
+  return launch_check();
+}
+
+template <typename T>
 cudaError_t prefill_simt_launch(const PrefillArgs& a, cudaStream_t st) {
   const int M = a.B * a.S, N = a.n_h * (a.d_h + a.d_v), K = a.d_c;
   // the expansion reads c_kv rows with their own stride; rows of different sequences are
@@ -370,7 +380,8 @@ cudaError_t prefill_simt_launch(const PrefillArgs& a, cudaStream_t st) {
   template cudaError_t out_up_simt_launch<T>(int, int, int, int, int, const void*, const void*, void*,    \
                                              cudaStream_t);                                           \
   template cudaError_t decode_simt_launch<T>(const DecodeArgs&, void*, cudaStream_t);                  \
-  template cudaError_t prefill_simt_launch<T>(const PrefillArgs&, cudaStream_t);
+  template cudaError_t prefill_simt_launch<T>(const PrefillArgs&, cudaStream_t);                    \
+  template cudaError_t prefill_attn_simt_launch<T>(const PrefillArgs&, cudaStream_t);
 
 MLA_INSTANTIATE(float)
 MLA_INSTANTIATE(__nv_bfloat16)
