@@ -29,6 +29,7 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st);
 cudaError_t absorb_q_tc_launch(int B, const void* q_nope, int64_t ldq, const void* w, void* q_tilde, cudaStream_t st);
 cudaError_t out_up_tc_launch(int B, const void* ctx, const void* w, void* out, cudaStream_t st);
 cudaError_t expand_tc_launch(const PrefillArgs& a, cudaStream_t st);
+cudaError_t attn_tc_launch(const PrefillArgs& a, cudaStream_t st);
 template <typename T>
 cudaError_t prefill_attn_simt_launch(const PrefillArgs& a, cudaStream_t st);
 size_t decode_static_scratch_bytes();

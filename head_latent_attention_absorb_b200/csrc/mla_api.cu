@@ -261,7 +261,7 @@ mla_status mla_prefill_naive(mla_dims dims, mla_dtype dtype, int32_t B, int32_t 
   if (dtype == MLA_BF16) {
     // tensor-core expansion (needs 16-byte-aligned rows for its TMA maps), then the attention
     e = mla::expand_tc_launch(a, st);
-    if (e == cudaSuccess) e = mla::prefill_attn_simt_launch<__nv_bfloat16>(a, st);
+    if (e == cudaSuccess) e = mla::attn_tc_launch(a, st);
   } else {
     e = mla::prefill_simt_launch<float>(a, st);
   }

@@ -232,6 +232,297 @@ __global__ void __launch_bounds__(kThreads, 1) expand_kernel(const __grid_consta
 size_t smem_bytes() { return (size_t)kBarOff + sizeof(Bars) + 1024; }
 static_assert(kBarOff + sizeof(Bars) + 1024 <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
 
+// ------------------------------------------------------------------------------------------
+// Causal attention of the naive path ("Naive path": k = [k_nope; k_R broadcast], scores
+// q . k / sqrt(192), softmax over positions t <= s, output sum_t alpha_t v_t), per (sequence,
+// head, 128-query tile):
+//   * Q (128 x 192) is TMA-loaded once and copied into TMEM (A operand of S = Q K^T);
+//   * K tiles (128 keys: k_nope from the expanded rows, k_R shared by the heads) and V tiles stream
+//     through a 2-stage TMA ring;
+//   * S goes to one of two TMEM buffers; the softmax (4 warps, one query row per thread) takes the
+//     row maximum, then writes P = 2^(s - m) as bf16 over the same columns, and P.V reads it from
+//     TMEM (A operand) while the next S is computed into the other buffer;
+//   * online softmax in base 2, the running maximum raised (and O rescaled) only when it grows by
+//     more than 8.
+// ------------------------------------------------------------------------------------------
+constexpr int AT_TILE = 128;                      // queries per CTA, keys per tile
+constexpr int AT_SLAB = AT_TILE * 128;            // 128 rows x 64 bf16 (128-byte swizzle)
+constexpr int AT_QOFF = 0;                        // Q: 3 slabs (q_nope 0-63, 64-127, q_pe)
+constexpr int AT_STAGE0 = 3 * AT_SLAB;            // stage: K slabs (k_nope x2, k_R) + V slabs x2
+constexpr int AT_STAGE_BYTES = 5 * AT_SLAB;
+constexpr int AT_STAGES = 2;
+constexpr int AT_BAROFF = AT_STAGE0 + AT_STAGES * AT_STAGE_BYTES;
+constexpr int AT_THREADS = 192;                   // warp 0 loads, warp 1 MMAs, warps 2-5 softmax
+constexpr uint32_t AT_COL_Q = 0, AT_COL_S = 128, AT_COL_O = 384;  // Q 96 cols, S 2 x 128, O 128
+
+struct AttnParams {
+  CUtensorMap tm_q;   // 4-D (192, H, S, B) query rows, box (64, 1, 128, 1)
+  CUtensorMap tm_kv;  // 4-D (256, H, S, B) expanded rows (k_nope | v), box (64, 1, 128, 1)
+  CUtensorMap tm_kr;  // 3-D (64, S, B) shared rotary keys, box (64, 128, 1)
+  __nv_bfloat16* out; // [B][S][H][128]
+  int B, S, H, n_qt, causal;
+  float scale_log2;
+  int32_t* err;
+};
+
+struct AttnBars {
+  uint64_t q_tma, q_full, full[AT_STAGES], empty[AT_STAGES], s_full[2], p_full[2], pv_done[2];
+  uint32_t tmem_base;
+  int abort;
+};
+
+__global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_constant__ AttnParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  AttnBars& bs = *reinterpret_cast<AttnBars*>(smem + AT_BAROFF);
+  volatile int* abort_flag = &bs.abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // the longest causal rows first: block 0 takes the last query tile of every (sequence, head)
+  const int idx = blockIdx.x;
+  const int h = idx % p.H, b = (idx / p.H) % p.B, qt = p.n_qt - 1 - idx / (p.H * p.B);
+  const int n_kv = p.causal ? qt + 1 : p.n_qt;   // key tiles this query tile attends
+
+  griddep_launch_dependents();
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bs.q_tma), 1);
+    mbar_init(smem_u32(&bs.q_full), 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&bs.full[i]), 1);
+      mbar_init(smem_u32(&bs.empty[i]), 1);
+      mbar_init(smem_u32(&bs.s_full[i]), 1);
+      mbar_init(smem_u32(&bs.p_full[i]), 4);
+      mbar_init(smem_u32(&bs.pv_done[i]), 1);
+    }
+    bs.abort = 0;
+    fence_mbar_init();
+    prefetch_tensormap(&p.tm_q);
+    prefetch_tensormap(&p.tm_kv);
+    prefetch_tensormap(&p.tm_kr);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bs.tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bs.tmem_base;
+  auto fail = [&]() {
+    raise_error(p.err, MLA_ERR_TIMEOUT);
+    bs.abort = 1;
+  };
+
+  if (warp == 0) {
+    // ---------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      griddep_wait();  // the expanded rows come from the preceding kernel
+      const uint64_t pol = policy_evict_last();
+      const uint32_t qb = smem_u32(&bs.q_tma);
+      mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
+      for (int sl = 0; sl < 3; ++sl)
+        tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * qt, b, pol);
+      bool ok = true;
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const uint32_t st = j % AT_STAGES, ph = (j / AT_STAGES) & 1u;
+        if (!mbar_wait(smem_u32(&bs.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
+          fail();
+          ok = false;
+          break;
+        }
+        const uint32_t dst = smem_u32(smem + AT_STAGE0 + st * AT_STAGE_BYTES);
+        const uint32_t bar = smem_u32(&bs.full[st]);
+        mbar_arrive_expect_tx(bar, AT_STAGE_BYTES);
+        tma_load_4d(dst, &p.tm_kv, bar, 0, h, AT_TILE * j, b, pol);                 // k_nope 0-63
+        tma_load_4d(dst + AT_SLAB, &p.tm_kv, bar, 64, h, AT_TILE * j, b, pol);      // k_nope 64-127
+        tma_load_3d(dst + 2 * AT_SLAB, &p.tm_kr, bar, 0, AT_TILE * j, b, pol);      // k_R
+        tma_load_4d(dst + 3 * AT_SLAB, &p.tm_kv, bar, 128, h, AT_TILE * j, b, pol); // v 0-63
+        tma_load_4d(dst + 4 * AT_SLAB, &p.tm_kv, bar, 192, h, AT_TILE * j, b, pol); // v 64-127
+      }
+      const int first = n_kv > AT_STAGES ? n_kv - AT_STAGES : 0;
+      for (int k = first; k < n_kv; ++k)
+        mbar_wait(smem_u32(&bs.full[k % AT_STAGES]), (k / AT_STAGES) & 1u, abort_flag, kWaitLimitNs);
+      mbar_wait(qb, 0, abort_flag, kWaitLimitNs);
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    const uint32_t idesc_qk = idesc_bf16_f32(128, AT_TILE, 0, 0);
+    const uint32_t idesc_pv = idesc_bf16_f32(128, 128, 0, 1);
+    bool ok = true;
+    auto wait_all = [&](uint32_t bar, uint32_t par) {
+      if (!ok) return false;
+      const bool mine = mbar_wait(bar, par, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, mine)) {
+        if (lane == 0) fail();
+        ok = false;
+      }
+      return ok;
+    };
+    auto issue_pv = [&](int j) {
+      if (!wait_all(smem_u32(&bs.p_full[j & 1]), (j >> 1) & 1u)) return;
+      tc_fence_after();
+      if (lane == 0) {
+        const uint32_t vb = smem_u32(smem + AT_STAGE0 + (j % AT_STAGES) * AT_STAGE_BYTES + 3 * AT_SLAB);
+        const uint32_t tP = tmem + AT_COL_S + 128 * (j & 1);
+#pragma unroll
+        for (int k = 0; k < AT_TILE / 16; ++k)
+          mma_ts(tmem + AT_COL_O, tP + 8 * k, smem_desc(vb + 2048 * k, AT_SLAB, 1024, kSwizzle128), idesc_pv,
+                 (j > 0 || k > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bs.empty[j % AT_STAGES]));
+        mma_commit(smem_u32(&bs.pv_done[j & 1]));
+      }
+      __syncwarp();
+    };
+    if (wait_all(smem_u32(&bs.q_full), 0)) {
+      tc_fence_after();
+      for (int j = 0; j < n_kv && ok; ++j) {
+        // S(j) = Q K(j)^T into buffer j & 1, free once P.V(j - 2) has read the P it held
+        if (!wait_all(smem_u32(&bs.full[j % AT_STAGES]), (j / AT_STAGES) & 1u)) break;
+        if (j >= 2 && !wait_all(smem_u32(&bs.pv_done[j & 1]), ((j - 2) >> 1) & 1u)) break;
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t kb = smem_u32(smem + AT_STAGE0 + (j % AT_STAGES) * AT_STAGE_BYTES);
+          const uint32_t tS = tmem + AT_COL_S + 128 * (j & 1);
+#pragma unroll
+          for (int k = 0; k < 12; ++k)  // 8 K-steps of q_nope . k_nope, 4 of q_pe . k_R
+            mma_ts(tS, tmem + AT_COL_Q + 8 * k, smem_desc(kb + (k >> 2) * AT_SLAB + 32 * (k & 3), 16, 1024, kSwizzle128),
+                   idesc_qk, k > 0 ? 1u : 0u);
+          mma_commit(smem_u32(&bs.s_full[j & 1]));
+        }
+        __syncwarp();
+        if (j >= 1) issue_pv(j - 1);  // P.V of the previous tile behind this tile's scores
+      }
+      if (ok && n_kv > 0) issue_pv(n_kv - 1);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax (warps 2-5)
+    const int quad = warp & 3;
+    const int r = 32 * quad + lane;               // query row of this thread within the tile
+    const int q_pos = AT_TILE * qt + r;           // its position in the sequence
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    const uint32_t tQ = tmem + lane_off + AT_COL_Q, tO = tmem + lane_off + AT_COL_O;
+    bool ok = true;
+    auto wait_all = [&](uint32_t bar, uint32_t par) {
+      if (!ok) return false;
+      const bool mine = mbar_wait(bar, par, abort_flag, kWaitLimitNs);
+      if (!__all_sync(0xffffffffu, mine)) {
+        if (lane == 0) fail();
+        ok = false;
+      }
+      return ok;
+    };
+    // Q row -> TMEM (A operand): 192 features as 96 columns of bf16 pairs
+    if (wait_all(smem_u32(&bs.q_tma), 0)) {
+      for (int sl = 0; sl < 3; ++sl) {
+        const uint32_t row = smem_u32(smem + AT_QOFF + sl * AT_SLAB) + r * 128;
+        uint32_t v[32];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 u = ld_shared_v4_b32(row + ((c ^ (r & 7)) << 4));
+          v[4 * c] = u.x; v[4 * c + 1] = u.y; v[4 * c + 2] = u.z; v[4 * c + 3] = u.w;
+        }
+        tmem_st32(tQ + 32 * sl, v);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bs.q_full));
+    }
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int j = 0; j < n_kv && ok; ++j) {
+      if (!wait_all(smem_u32(&bs.s_full[j & 1]), (j >> 1) & 1u)) break;
+      tc_fence_after();
+      const uint32_t tS = tmem + lane_off + AT_COL_S + 128 * (j & 1);
+      const int key0 = AT_TILE * j;
+      // keys of this tile this row may attend: below the sequence length and (causal) <= q_pos
+      const int lim = p.causal ? min(p.S - 1, q_pos) : p.S - 1;
+      const int nvalid = lim - key0 + 1;  // keys 0 .. nvalid-1 of the tile are valid
+      float mx = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tS + 32 * c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          if (32 * c + k < nvalid) mx = fmaxf(mx, __uint_as_float(v[k]));
+      }
+      const float m_new = fmaxf(m_run, mx * p.scale_log2);
+      const bool need = m_new > m_run + 8.0f;  // true on the first tile (m_run = -inf)
+      if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // O holds P.V of the earlier tiles relative to the old maximum: rescale it once the
+        // last of those products has landed
+        if (!wait_all(smem_u32(&bs.pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1u)) break;
+        tc_fence_after();
+        const float corr = need ? ex2f_approx(m_run - m_new) : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tO + 32 * c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * corr);
+          tmem_st32(tO + 32 * c, v);
+        }
+      }
+      if (need) {
+        l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2f_approx(m_run - m_new);
+        m_run = m_new;
+      }
+      // P = 2^(s scale_log2 - m) in bf16, written over the scores it came from (chunk c of P takes
+      // columns [16c, 16c + 16), all already read)
+      float ls = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32], pk[16];
+        tmem_ld32(tS + 32 * c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int k0 = 32 * c + 2 * k;
+          const float p0 = k0 < nvalid ? ex2f_approx(fmaf(__uint_as_float(v[2 * k]), p.scale_log2, -m_run)) : 0.f;
+          const float p1 = k0 + 1 < nvalid ? ex2f_approx(fmaf(__uint_as_float(v[2 * k + 1]), p.scale_log2, -m_run)) : 0.f;
+          ls += p0 + p1;
+          pk[k] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(tS + 16 * c, pk);
+      }
+      l_run += ls;
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bs.p_full[j & 1]));
+    }
+    // ---- epilogue: O / l -> out (P.V of the last two tiles, older first)
+    if (ok && n_kv >= 2) wait_all(smem_u32(&bs.pv_done[(n_kv - 2) & 1]), ((n_kv - 2) >> 1) & 1u);
+    if (ok && n_kv >= 1 && wait_all(smem_u32(&bs.pv_done[(n_kv - 1) & 1]), ((n_kv - 1) >> 1) & 1u)) {
+      tc_fence_after();
+      const float inv = 1.f / l_run;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + 32 * c, v);
+        tmem_ld_wait();
+        if (q_pos < p.S) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + (((int64_t)b * p.S + q_pos) * p.H + h) * 128 + 32 * c);
+#pragma unroll
+          for (int w = 0; w < 4; ++w)
+            dst[w] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * w]) * inv, __uint_as_float(v[8 * w + 1]) * inv),
+                                pack_bf16x2(__uint_as_float(v[8 * w + 2]) * inv, __uint_as_float(v[8 * w + 3]) * inv),
+                                pack_bf16x2(__uint_as_float(v[8 * w + 4]) * inv, __uint_as_float(v[8 * w + 5]) * inv),
+                                pack_bf16x2(__uint_as_float(v[8 * w + 6]) * inv, __uint_as_float(v[8 * w + 7]) * inv));
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+size_t attn_smem_bytes() { return (size_t)AT_BAROFF + sizeof(AttnBars) + 1024; }
+static_assert(AT_BAROFF + sizeof(AttnBars) + 1024 <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
 }  // namespace prefill_tc
 
 // kv[B*S, n_h*(d_h+d_v)] = c_kv[B*S, d_c] * w_kv_b^T, bf16, DeepSeek dimensions.
@@ -271,6 +562,45 @@ cudaError_t expand_tc_launch(const PrefillArgs& a, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(expand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(expand_kernel, dim3(grid), dim3(kThreads), smem, st, p);
+}
+
+// Causal (or full) attention of the naive path over the expanded rows in a.kv, bf16, DeepSeek dims.
+cudaError_t attn_tc_launch(const PrefillArgs& a, cudaStream_t st) {
+  using namespace prefill_tc;
+  AttnParams p;
+  memset(&p, 0, sizeof(p));
+  const uint64_t H = (uint64_t)a.n_h, S = (uint64_t)a.S, B = (uint64_t)a.B;
+  const uint64_t dq = (uint64_t)(a.d_h + a.d_r), dkv = (uint64_t)(a.d_h + a.d_v);
+  {
+    const uint64_t dims[4] = {dq, H, S, B}, strides[3] = {dq * 2, H * dq * 2, S * H * dq * 2};
+    const uint32_t box[4] = {64, 1, AT_TILE, 1};
+    if (!make_tensor_map_bf16(&p.tm_q, a.q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[4] = {dkv, H, S, B}, strides[3] = {dkv * 2, H * dkv * 2, S * H * dkv * 2};
+    const uint32_t box[4] = {64, 1, AT_TILE, 1};
+    if (!make_tensor_map_bf16(&p.tm_kv, a.kv, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)a.d_r, S, B}, strides[2] = {(uint64_t)a.kr_r * 2, S * (uint64_t)a.kr_r * 2};
+    const uint32_t box[3] = {64, AT_TILE, 1};
+    if (!make_tensor_map_bf16(&p.tm_kr, a.k_r, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+      return cudaErrorInvalidValue;
+  }
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.B = a.B;
+  p.S = a.S;
+  p.H = a.n_h;
+  p.n_qt = (a.S + AT_TILE - 1) / AT_TILE;
+  p.causal = a.causal;
+  p.scale_log2 = a.scale * 1.4426950408889634f;
+  p.err = nullptr;
+  const size_t smem = attn_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(attn_kernel, dim3((unsigned)(p.n_qt * a.B * a.n_h)), dim3(AT_THREADS), smem, st, p);
 }
 
 }  // namespace mla
