@@ -1262,8 +1262,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                  acc[8 * v + 2 * q] = w_own * own_v[8 * v + 2 * q] + w_other * bf16_lo(uw[q]);
-                  acc[8 * v + 2 * q + 1] = w_own * own_v[8 * v + 2 * q + 1] + w_other * bf16_hi(uw[q]);
+                  // both products rounded on their own (no fused multiply-add), so the sum is the
+                  // same whichever of the two clusters merges
+                  acc[8 * v + 2 * q] = __fadd_rn(__fmul_rn(w_own, own_v[8 * v + 2 * q]), __fmul_rn(w_other, bf16_lo(uw[q])));
+                  acc[8 * v + 2 * q + 1] =
+                      __fadd_rn(__fmul_rn(w_own, own_v[8 * v + 2 * q + 1]), __fmul_rn(w_other, bf16_hi(uw[q])));
                 }
               }
             } else {
