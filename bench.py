@@ -165,7 +165,7 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def time_secondary(dev, reps: int):
+def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill")):
     """The other workloads of the hot path, each timed on its own with CUDA events (L2 flushed
     before every launch): the ragged long-context decode, the V3.2 top-k decode and the naive causal
     prefill.  Reported beside the headline line; algorithmic bytes / FLOPs as for the headline."""
@@ -185,7 +185,7 @@ def time_secondary(dev, reps: int):
         return statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev[3:])
 
     out = {}
-    for cfg in (RAGGED_LONG, SPARSE_V32):
+    for cfg in [c for c, k in ((RAGGED_LONG, "ragged"), (SPARSE_V32, "sparse")) if k in which]:
         x = make_decode_inputs(cfg)
         cache = x["cache"].to(dev)
         c_kv, k_r = cache[..., :cfg.d_c], cache[..., cfg.d_c:]
@@ -210,6 +210,8 @@ def time_secondary(dev, reps: int):
                          "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": flops / (ms * 1e-3) / 1e12}
         del x, cache, c_kv, k_r, ws
         torch.cuda.empty_cache()
+    if "prefill" not in which:
+        return out
     cfg = PREFILL
     p = make_prefill_inputs(cfg)
     q, c_kv, k_r, w = p["q"].to(dev), p["c_kv"].to(dev), p["k_r"].to(dev), p["w_kv_b"].to(dev)
@@ -389,8 +391,16 @@ def main():
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the timings of the ragged, top-k and prefill workloads")
+    ap.add_argument("--only", choices=["ragged", "sparse", "prefill"],
+                    help="time only this secondary workload (--steps launches after 3 warm-up ones) and print "
+                         "its entry; a small command for profilers, not a bench line")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.only:
+        dev = torch.device("cuda", 0)
+        torch.cuda.set_device(dev)
+        print(json.dumps(time_secondary(dev, args.steps, (args.only,))))
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -111,6 +111,7 @@ struct Smem {
   uint64_t pub_bar, last_bar;      // partial published by all softmax warps / merge decision made
   uint64_t mrg_full;               // the other cluster's partial bulk-loaded for the merge
   uint64_t mrg_full2[2], mrg_empty2[2];  // streamed merge of several partials (double-buffered)
+  uint64_t xch_drained;            // the peer has read every partial score this CTA sent
   float red[2][2][kNH];            // [tile parity][key half][head] partial row max
   float lsum[2][kNH];              // [key half][head] partial softmax sum
   int16_t slots[kMaxClusters];     // partial slots of the sequence being merged
@@ -481,6 +482,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&sm.pub_bar), kSoftmaxWarps);
     mbar_init(smem_u32(&sm.last_bar), 1);
     mbar_init(smem_u32(&sm.mrg_full), 1);
+    mbar_init(smem_u32(&sm.xch_drained), 4);  // the four exchange warps
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.mrg_full2[i]), 1);
       mbar_init(smem_u32(&sm.mrg_empty2[i]), kSoftmaxWarps);
@@ -536,7 +538,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           q_issued = true;
         }
         const int seq_len_b = p.topk > 0 ? clamp_len(p.lengths[b], p.n_max) : 0;
+        // sparse: the positions of tile i + 1 are loaded while tile i is issued (two per lane), so
+        // no tile waits for its own index load
+        int pos_next[2] = {0, 0};
+        auto load_pos = [&](int i, int (&dst)[2]) {
+#pragma unroll
+          for (int hf = 0; hf < 2; ++hf) {
+            const int k = i * kTile + 32 * hf + lane;
+            dst[hf] = k < p.topk ? p.topk_idx[(int64_t)b * p.topk + k] : 0;
+          }
+        };
+        if (p.topk > 0) load_pos(begin, pos_next);
         for (int i = begin; i < end && ok; ++i, ++it) {
+          int pos_cur[2] = {pos_next[0], pos_next[1]};
+          if (p.topk > 0 && i + 1 < end) load_pos(i + 1, pos_next);
           const uint32_t st = it % kStages, ph = (it / kStages) & 1u;
           if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs))) {
             if (lane == 0) fail_timeout(sm, p.err);
@@ -559,10 +574,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int rows[2];
 #pragma unroll
             for (int hf = 0; hf < 2; ++hf) {
-              const int k = i * kTile + 32 * hf + lane;
               int pos = 0;
-              if (k < p.topk) {
-                pos = p.topk_idx[(int64_t)b * p.topk + k];
+              if (i * kTile + 32 * hf + lane < p.topk) {
+                pos = pos_cur[hf];
                 if (pos < 0 || pos >= seq_len_b) {
                   raise_error(p.err, MLA_ERR_INDEX);
                   pos = 0;
@@ -777,6 +791,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         mbar_arrive(smem_u32(&sm.own_ready[xi]));
       }
     }
+    // Once the peer has read the last two partials this CTA sent, no copy reads the staging buffers
+    // any more and the exchange buffers may hold other data (the split-KV merge).  The peer's read
+    // of tile t completes phase (t >> 1) + 1 of x_free[t & 1].
+    for (uint32_t t = ntiles >= 2 ? ntiles - 2 : 0; t < ntiles && ok; ++t)
+      wait_or_fail(smem_u32(&sm.x_free[t & 1u]), ((t >> 1) + 1u) & 1u, true);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_u32(&sm.xch_drained));
   } else {
     // ------------------------------------------------------------------ softmax warps (kBWarp0..)
     griddep_wait();  // they read the absorbed query and write the context / workspace
@@ -1066,7 +1087,92 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           for (int i = 0; i < ns; ++i)
             if (sm.slots[i] != own) other = sm.slots[i];
           const bool bulk = (ns == 2) && (base + end >= sm.hi);
-          if (ns > 2 && base + end >= sm.hi) {
+          if (ns > 2 && (ns - 1) * 65536 <= kSmemOff && base + end >= sm.hi) {
+            // ---- up to three other partials, and no further cache tiles will land in the stage
+            // buffers: all of them are bulk-loaded at once into the free stage / exchange buffers
+            // (64 KB each) and merged in registers, in slot order with the arithmetic of the
+            // streamed merge below (same result bit for bit); this CTA's own partial is read from
+            // its O columns, normalised and rounded through bf16 like a published one.
+            // a third partial goes into the exchange buffers: wait until they are quiet
+            if (ns - 1 > 2 && !wait_or_fail(smem_u32(&sm.xch_drained), 0, false)) break;
+            if (sw == 0 && lane == 0) {
+              fence_proxy_async_global();  // the partials were written through the generic proxy
+              const uint32_t bar = smem_u32(&sm.mrg_full);
+              mbar_arrive_expect_tx(bar, (uint32_t)(ns - 1) * kNH * 512);
+              int k = 0;
+              for (int i = 0; i < ns; ++i) {
+                const int sl = sm.slots[i];
+                if (sl == own) continue;
+                const uint8_t* src = reinterpret_cast<const uint8_t*>(p.ws_o) + ((int64_t)sl * 2 + rank) * kNH * 512;
+                const uint32_t dst = smem_u32(smem) + (uint32_t)k * 65536u;
+                bulk_load_g2s(dst, src, 32768, bar);
+                bulk_load_g2s(dst + 32768, src + 32768, 32768, bar);
+                ++k;
+              }
+            }
+            float M = m_run;
+            for (int i = 0; i < ns; ++i)
+              if (sm.slots[i] != own) M = fmaxf(M, __ldcg(p.ws_ml + ((int64_t)sm.slots[i] * 2 + rank) * kNH + h).x);
+            float L = 0.f;
+            for (int i = 0; i < ns; ++i) {
+              const int sl = sm.slots[i];
+              const float2 ml = sl == own ? make_float2(m_run, l_tot) : __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
+              L += ml.y * ex2(ml.x - M);
+            }
+            const float inv = 1.f / L;
+            if (!wait_or_fail(smem_u32(&sm.mrg_full), nmrg & 1u, false)) break;
+            ++nmrg;
+            __nv_bfloat16* dst = p.ctx + ((int64_t)b * kNH + h) * kDC + 256 * rank + 128 * half;
+#pragma unroll 1
+            for (int c = 0; c < 4; ++c) {
+              uint32_t r[32];
+              tmem_ld32(tO + c * 32, r);
+              tmem_ld_wait();
+              uint32_t ow[16];
+#pragma unroll
+              for (int k = 0; k < 16; ++k)
+                ow[k] = pack_bf16x2(__uint_as_float(r[2 * k]) * inv_own, __uint_as_float(r[2 * k + 1]) * inv_own);
+              float acc[32];
+#pragma unroll
+              for (int q = 0; q < 32; ++q) acc[q] = 0.f;
+              int k = 0;
+              for (int i = 0; i < ns; ++i) {
+                const int sl = sm.slots[i];
+                uint32_t uw[16];
+                float w;
+                if (sl == own) {
+                  w = l_tot * ex2(m_run - M) * inv;
+#pragma unroll
+                  for (int q = 0; q < 16; ++q) uw[q] = ow[q];
+                } else {
+                  const float2 ml = __ldcg(p.ws_ml + ((int64_t)sl * 2 + rank) * kNH + h);
+                  w = ml.y * ex2(ml.x - M) * inv;
+                  const uint4* srow = reinterpret_cast<const uint4*>(smem + (size_t)k * 65536) + h * 32;
+#pragma unroll
+                  for (int v = 0; v < 4; ++v) {
+                    const uint4 u = srow[(16 * half + 4 * c + v) ^ cswz];
+                    uw[4 * v] = u.x; uw[4 * v + 1] = u.y; uw[4 * v + 2] = u.z; uw[4 * v + 3] = u.w;
+                  }
+                  ++k;
+                }
+#pragma unroll
+                for (int q = 0; q < 16; ++q) {
+                  acc[2 * q] = fmaf(w, bf16_lo(uw[q]), acc[2 * q]);
+                  acc[2 * q + 1] = fmaf(w, bf16_hi(uw[q]), acc[2 * q + 1]);
+                }
+              }
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
+                                   pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+            }
+            if (rank == 0 && half == 0 && p.lse != nullptr)
+              p.lse[(int64_t)b * kNH + h] = (M + log2f(L)) * 0.69314718055994531f;
+            if (sw == 0 && lane == 0)
+              for (int i = 0; i < ns; ++i)
+                if (sm.slots[i] != own) p.ws_ready[2 * (int64_t)sm.slots[i] + rank] = 0ull;
+          } else if (ns > 2 && base + end >= sm.hi) {
             // ---- several partials, and no further cache tiles will land in the stage buffers:
             // stream the other partials through two 64 KB stage buffers (bulk loads, one ahead),
             // accumulating in TMEM in slot order.  This CTA's own partial, normalised and rounded

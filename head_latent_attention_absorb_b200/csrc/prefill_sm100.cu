@@ -277,9 +277,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
   AttnBars& bs = *reinterpret_cast<AttnBars*>(smem + AT_BAROFF);
   volatile int* abort_flag = &bs.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // the longest causal rows first: block 0 takes the last query tile of every (sequence, head)
+  // The query tiles of one (sequence, head) are consecutive blocks, the longest causal rows first:
+  // blocks that run together share that head's K/V tiles in L2 (read from HBM about once), and
+  // the short tiles of a head free their SMs early for the next head's long ones.
   const int idx = blockIdx.x;
-  const int h = idx % p.H, b = (idx / p.H) % p.B, qt = p.n_qt - 1 - idx / (p.H * p.B);
+  const int qt = p.n_qt - 1 - idx % p.n_qt, h = (idx / p.n_qt) % p.H, b = idx / (p.n_qt * p.H);
   const int n_kv = p.causal ? qt + 1 : p.n_qt;   // key tiles this query tile attends
 
   griddep_launch_dependents();
