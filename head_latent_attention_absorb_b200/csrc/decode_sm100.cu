@@ -64,6 +64,7 @@ constexpr int kXOff = kStages * kStageBytes;    // shared-memory layout: stages 
 constexpr int kQRopeOff = kXOff + 4 * kXBytes;
 constexpr int kSmemOff = kQRopeOff + kQRopeBytes;
 constexpr int kMaxClusters = 160;               // partial-slot list capacity (2 slots per cluster)
+constexpr int kMergeLastMax = 4;                // up to this many partials the last cluster merges alone
 constexpr int kSoftmaxWarps = 8;                // two per TMEM lane quadrant
 constexpr int kPvWarp = 2;                      // the warp that issues the P*V MMAs
 constexpr int kAWarp0 = 3;                      // 4 exchange warps, one per TMEM lane quadrant
@@ -112,6 +113,7 @@ struct Smem {
   uint64_t mrg_full;               // the other cluster's partial bulk-loaded for the merge
   uint64_t mrg_full2[2], mrg_empty2[2];  // streamed merge of several partials (double-buffered)
   uint64_t xch_drained;            // the peer has read every partial score this CTA sent
+  uint64_t mrg_done;               // every softmax warp finished its share of a sliced merge
   float red[2][2][kNH];            // [tile parity][key half][head] partial row max
   float lsum[2][kNH];              // [key half][head] partial softmax sum
   int16_t slots[kMaxClusters];     // partial slots of the sequence being merged
@@ -399,7 +401,16 @@ __device__ int list_slots(const Params& p, Smem& sm, int base, int nt) {
 // initialisation.  Every failed compare-and-swap means another CTA's arrival succeeded, so the
 // loop ends after at most `expected` rounds; the bound is only a guard.
 __device__ bool arrive_last(unsigned long long* ctr, unsigned long long epoch, int expected, int32_t* err) {
-  unsigned long long cur = 0;  // the value the previous launch's last arrival leaves
+  // Fast path, one or two atomics: the counter is 0 (left so by the previous launch's last arrival)
+  // or already tagged with this launch's epoch (then adding 1 keeps the tag: arrivals < 256).
+  unsigned long long cur = atomicCAS(ctr, 0ull, (epoch << 8) | 1ull);
+  if (cur == 0ull || (cur >> 8) == epoch) {
+    const unsigned long long now = cur == 0ull ? ((epoch << 8) | 1ull) : atomicAdd(ctr, 1ull) + 1ull;
+    if ((int)(now & 255ull) < expected) return false;
+    atomicExch(ctr, 0ull);  // every arrival of this launch is in: leave the counter for the next one
+    return true;
+  }
+  // a counter another launch left behind (it stopped early): tag it with a compare-and-swap loop
   for (int i = 0; i < 4096; ++i) {
     const unsigned long long base = (cur >> 8) == epoch ? cur : (epoch << 8);
     const unsigned long long next = base + 1;
@@ -483,6 +494,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     mbar_init(smem_u32(&sm.last_bar), 1);
     mbar_init(smem_u32(&sm.mrg_full), 1);
     mbar_init(smem_u32(&sm.xch_drained), 4);  // the four exchange warps
+    mbar_init(smem_u32(&sm.mrg_done), kSoftmaxWarps);
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.mrg_full2[i]), 1);
       mbar_init(smem_u32(&sm.mrg_empty2[i]), kSoftmaxWarps);
@@ -822,7 +834,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     int b, begin, end, len, base;
     bool whole;
     uint32_t tb = 0;           // global tile counter
-    uint32_t nseg = 0, npart = 0, npub = 0, nmrg = 0;
+    uint32_t nseg = 0, npart = 0, npub = 0, nmrg = 0, nmd = 0;
     bool ok = true;
     bool first_seg = true;     // the first segment of the range uses partial slot 2c, the last 2c + 1
     auto wait_or_fail = [&](uint32_t bar, uint32_t par, bool cl_scope) {
@@ -1026,7 +1038,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int own = 2 * cl + (first_seg ? 0 : 1);
         if (sw == 0 && lane == 0) {
           const int ns = list_slots(p, sm, base, tiles_of(len));
-          sm.is_last = arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0;
+          // up to kMergeLastMax partials the last cluster to arrive merges them all; with more, every
+          // cluster publishes and then merges its own slice of the heads
+          sm.is_last = ns > kMergeLastMax ? 0 : (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0);
           mbar_arrive(smem_u32(&sm.last_bar));
         }
         if (!wait_or_fail(smem_u32(&sm.last_bar), npart & 1u, false)) break;
@@ -1066,7 +1080,73 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
           }
           ++npub;
-        } else {
+        }
+        if (sm.nslots > kMergeLastMax) {
+          // ---- sliced merge: every slot's partial is published (lane 0 of each warp polls the flags,
+          // this cluster's own included); this CTA merges heads [h_lo, h_hi) of its latent half, one
+          // head per warp and one 16-byte chunk per lane, summing the slots in slot order.  The last
+          // cluster to finish its slice resets the flags for the next launch.
+          const int ns = sm.nslots;
+          int okw = 1;
+          if (lane == 0) {
+            for (int i = 0; i < ns && okw; ++i)
+              okw = wait_flag(p.ws_ready + 2 * (int64_t)sm.slots[i] + rank, p.epoch, abort_flag) ? 1 : 0;
+            if (!okw) fail_timeout(sm, p.err);
+          }
+          if (!__shfl_sync(0xffffffffu, okw, 0)) {
+            ok = false;
+            break;
+          }
+          int pos = 0;
+          for (int i = 0; i < ns; ++i)
+            if (sm.slots[i] == own) pos = i;
+          const int h_lo = pos * kNH / ns, h_hi = (pos + 1) * kNH / ns;
+          for (int hh = h_lo + sw; hh < h_hi; hh += kSoftmaxWarps) {
+            const float2* mlp = p.ws_ml + rank * kNH + hh;  // + slot * 2 * kNH
+            float M = -INFINITY;
+#pragma unroll 4
+            for (int i = 0; i < ns; ++i) M = fmaxf(M, __ldcg(mlp + (int64_t)sm.slots[i] * 2 * kNH).x);
+            float L = 0.f;
+#pragma unroll 4
+            for (int i = 0; i < ns; ++i) {
+              const float2 ml = __ldcg(mlp + (int64_t)sm.slots[i] * 2 * kNH);
+              L += ml.y * ex2(ml.x - M);
+            }
+            const float inv = 1.f / L;
+            float acc[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+            const uint4* base4 = reinterpret_cast<const uint4*>(p.ws_o) + ((int64_t)rank * kNH + hh) * 32 + (lane ^ (hh & 15));
+#pragma unroll 4
+            for (int i = 0; i < ns; ++i) {
+              const int64_t sl = sm.slots[i];
+              const float2 ml = __ldcg(mlp + sl * 2 * kNH);
+              const float w = ml.y * ex2(ml.x - M) * inv;
+              const uint4 u = __ldcg(base4 + sl * 2 * kNH * 32);
+              const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                acc[2 * q] = fmaf(w, bf16_lo(uw[q]), acc[2 * q]);
+                acc[2 * q + 1] = fmaf(w, bf16_hi(uw[q]), acc[2 * q + 1]);
+              }
+            }
+            *reinterpret_cast<uint4*>(p.ctx + ((int64_t)b * kNH + hh) * kDC + 256 * rank + 8 * lane) =
+                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                           pack_bf16x2(acc[6], acc[7]));
+            if (rank == 0 && lane == 0 && p.lse != nullptr)
+              p.lse[(int64_t)b * kNH + hh] = (M + log2f(L)) * 0.69314718055994531f;
+          }
+          warp_arrive(smem_u32(&sm.mrg_done));
+          if (sw == 0 && lane == 0) {
+            if (mbar_wait(smem_u32(&sm.mrg_done), nmd & 1u, abort_flag, kWaitLimitNs)) {
+              if (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err))
+                for (int i = 0; i < ns; ++i) p.ws_ready[2 * (int64_t)sm.slots[i] + rank] = 0ull;
+            } else {
+              fail_timeout(sm, p.err);
+            }
+          }
+          ++nmd;
+        } else if (sm.is_last) {
           const int ns = sm.nslots;
           // every other slot's partial has been published (lane 0 of each warp polls the flags)
           int okw = 1;
