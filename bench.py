@@ -37,7 +37,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch on this workload,
 # from the ncu capture summarised in profiles/decode_kernel_v3_b32_n4096.md, valid only for the
 # kernel source it was taken on (sha256 prefix of csrc/decode_sm100.cu).
-DECODE_TRAFFIC = {"bytes": 155_826_944 + 3_242_496, "source_sha256": "fb201eaa41de3b52"}
+DECODE_TRAFFIC = {"bytes": 155_848_960 + 7_039_232, "source_sha256": "af96b1671f600577"}
 
 
 def decode_traffic():
