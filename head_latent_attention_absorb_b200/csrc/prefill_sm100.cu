@@ -438,16 +438,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       // keys of this tile this row may attend: below the sequence length and (causal) <= q_pos
       const int lim = p.causal ? min(p.S - 1, q_pos) : p.S - 1;
       const int nvalid = lim - key0 + 1;  // keys 0 .. nvalid-1 of the tile are valid
+      // the whole score row in registers: four loads, one wait (the row is read from TMEM once)
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
+      tmem_ld_wait();
       float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + 32 * c, v);
-        tmem_ld_wait();
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int k = 0; k < 32; ++k)
-          if (32 * c + k < nvalid) mx = fmaxf(mx, __uint_as_float(v[k]));
-      }
+          if (32 * c + k < nvalid) mx = fmaxf(mx, __uint_as_float(sv[c][k]));
       const float m_new = fmaxf(m_run, mx * p.scale_log2);
       const bool need = m_new > m_run + 8.0f;  // true on the first tile (m_run = -inf)
       if (j > 0 && __any_sync(0xffffffffu, need)) {
@@ -471,18 +472,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
         m_run = m_new;
       }
       // P = 2^(s scale_log2 - m) in bf16, written over the scores it came from (chunk c of P takes
-      // columns [16c, 16c + 16), all already read)
+      // columns [16c, 16c + 16); the whole row is already in registers)
       float ls = 0.f;
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t v[32], pk[16];
-        tmem_ld32(tS + 32 * c, v);
-        tmem_ld_wait();
+        uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           const int k0 = 32 * c + 2 * k;
-          const float p0 = k0 < nvalid ? ex2f_approx(fmaf(__uint_as_float(v[2 * k]), p.scale_log2, -m_run)) : 0.f;
-          const float p1 = k0 + 1 < nvalid ? ex2f_approx(fmaf(__uint_as_float(v[2 * k + 1]), p.scale_log2, -m_run)) : 0.f;
+          const float p0 = k0 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k]), p.scale_log2, -m_run)) : 0.f;
+          const float p1 = k0 + 1 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k + 1]), p.scale_log2, -m_run)) : 0.f;
           ls += p0 + p1;
           pk[k] = pack_bf16x2(p0, p1);
         }
