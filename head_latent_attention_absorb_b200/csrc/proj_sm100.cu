@@ -9,9 +9,11 @@
 // N (padded to a multiple of 16, at most 256 per CTA):
 //   absorb_q: D[c, b] = W^UK_h^T[c, d] q_nope_h^T[d, b]   A = W^UK_h read MN-major, K = 128
 //   out_up:   D[d, b] = W^UV_h[d, c]   ctx_h^T[c, b]      A = W^UV_h read K-major,  K = 512
-// One CTA computes one (head, 128-row block, batch block) tile: TMA brings the W block and the
+// One CTA computes the tiles of one (head, batch block) and kMB 128-row blocks (two for absorb_q,
+// whose four latent blocks of a head share the activations): TMA brings the W blocks and the
 // activations (K split in 64-wide chunks, one mbarrier each, so MMAs start on the first chunk),
-// one thread issues the MMAs, and the four warps read the accumulator back from TMEM.
+// one thread issues the MMAs into one TMEM accumulator per block, and four warps per block read
+// them back.  Fewer, larger CTAs start sooner (the launch of 512 small ones took ~2 us).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <string.h>
@@ -41,17 +43,19 @@ template <bool kAbsorb>
 struct Shape {
   static constexpr int kChunks = kAbsorb ? kDH / 64 : kDC / 64;       // 64-wide K chunks
   static constexpr int kAChunkBytes = 128 * 64 * 2;                   // 128 M rows x 64 K
+  static constexpr int kMB = kAbsorb ? 2 : 1;                         // 128-row blocks per CTA
+  static constexpr int kThreads = 128 * kMB;                          // four epilogue warps per block
 };
 
 __device__ __forceinline__ uint32_t tmem_cols_for(int n) { return n <= 32 ? 32 : (n <= 64 ? 64 : (n <= 128 ? 128 : 256)); }
 
 template <bool kAbsorb>
-__global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Params p) {
+__global__ void __launch_bounds__(Shape<kAbsorb>::kThreads) proj_kernel(const __grid_constant__ Params p) {
   using S = Shape<kAbsorb>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* a_s = smem;                                     // kChunks x 16 KB
-  uint8_t* b_s = smem + S::kChunks * S::kAChunkBytes;      // kChunks x (n_tile x 128 B)
+  uint8_t* a_s = smem;                                          // [kMB][kChunks] x 16 KB
+  uint8_t* b_s = smem + S::kMB * S::kChunks * S::kAChunkBytes;  // kChunks x (n_tile x 128 B)
   __shared__ uint64_t full[S::kChunks];
   __shared__ uint64_t done;
   __shared__ uint32_t tmem_base;
@@ -59,7 +63,7 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
-  const int m0 = kAbsorb ? blockIdx.x * 128 : 0;   // first latent feature (absorb_q) of this CTA
+  const int m0 = kAbsorb ? blockIdx.x * 128 * S::kMB : 0;  // first latent feature (absorb_q) of this CTA
   const int b0 = blockIdx.z * p.n_tile;
   const int n = p.n_tile;
   const uint32_t ncols = tmem_cols_for(n);
@@ -75,7 +79,7 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
     prefetch_tensormap(&p.tm_act);
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(&tmem_base), ncols);
+    tmem_alloc(smem_u32(&tmem_base), ncols * S::kMB);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -89,13 +93,17 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
     // the weights are no kernel's output: load them before waiting for the preceding kernel
     for (int j = 0; j < S::kChunks; ++j) {
       const uint32_t bar = smem_u32(&full[j]);
-      mbar_arrive_expect_tx(bar, S::kAChunkBytes + b_chunk_bytes);
+      mbar_arrive_expect_tx(bar, S::kMB * S::kAChunkBytes + b_chunk_bytes);
       const uint32_t a_dst = smem_u32(a_s + j * S::kAChunkBytes);
       if (kAbsorb) {
-        // W^UK_h rows d in [64 j, 64 j + 64), latent columns [m0, m0 + 128) as two 64-column boxes:
-        // MN-major A (M = latent feature contiguous), one 8 KB box per 64 M values
-        tma_load_2d(a_dst, &p.tm_w, bar, m0, h * kRowsPerHead + 64 * j, pol_w);
-        tma_load_2d(a_dst + 8192, &p.tm_w, bar, m0 + 64, h * kRowsPerHead + 64 * j, pol_w);
+        // W^UK_h rows d in [64 j, 64 j + 64), latent columns [m0 + 128 mb, + 128) as two 64-column
+        // boxes per block: MN-major A (M = latent feature contiguous), one 8 KB box per 64 M values
+#pragma unroll
+        for (int mb = 0; mb < S::kMB; ++mb) {
+          const uint32_t d = a_dst + mb * S::kChunks * S::kAChunkBytes;
+          tma_load_2d(d, &p.tm_w, bar, m0 + 128 * mb, h * kRowsPerHead + 64 * j, pol_w);
+          tma_load_2d(d + 8192, &p.tm_w, bar, m0 + 128 * mb + 64, h * kRowsPerHead + 64 * j, pol_w);
+        }
       } else {
         // W^UV_h rows d in [0, 128), latent columns [64 j, 64 j + 64): K-major A
         tma_load_2d(a_dst, &p.tm_w, bar, 64 * j, h * kRowsPerHead + kDH, pol_w);
@@ -115,13 +123,17 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
         break;
       }
       tc_fence_after();
-      const uint32_t a_base = smem_u32(a_s + j * S::kAChunkBytes), b_base = smem_u32(b_s + j * b_chunk_bytes);
+      const uint32_t b_base = smem_u32(b_s + j * b_chunk_bytes);
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t ad = kAbsorb ? smem_desc(a_base + kk * 2048, 8192, 1024, kSwizzle128)   // 16 K rows
-                                    : smem_desc(a_base + kk * 32, 16, 1024, kSwizzle128);      // 16 K columns
-        const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, kSwizzle128);
-        mma_ss(tmem, ad, bd, idesc, (j | kk) ? 1u : 0u);
+      for (int mb = 0; mb < S::kMB; ++mb) {
+        const uint32_t a_base = smem_u32(a_s + (mb * S::kChunks + j) * S::kAChunkBytes);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t ad = kAbsorb ? smem_desc(a_base + kk * 2048, 8192, 1024, kSwizzle128)   // 16 K rows
+                                      : smem_desc(a_base + kk * 32, 16, 1024, kSwizzle128);      // 16 K columns
+          const uint64_t bd = smem_desc(b_base + kk * 32, 16, 1024, kSwizzle128);
+          mma_ss(tmem + mb * ncols, ad, bd, idesc, (j | kk) ? 1u : 0u);
+        }
       }
     }
     mma_commit(smem_u32(&done));
@@ -129,15 +141,17 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
   }
   __syncwarp();
 
-  // ---- epilogue: lane i of warp w holds row 32 w + i of D (a latent feature / value feature)
+  // ---- epilogue: lane i of warp w holds row 32 (w % 4) + i of block w / 4 of D (a latent /
+  // value feature)
   griddep_wait();  // every thread that writes the output waits for the preceding kernel
   const bool ok = mbar_wait(smem_u32(&done), 0, &abort_flag, kWaitLimitNs);
   if (__all_sync(0xffffffffu, ok)) {
     tc_fence_after();
-    const int row = 32 * warp + lane;
-    const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16);
+    const int mb = warp >> 2, quad = warp & 3;
+    const int row = 32 * quad + lane;
+    const uint32_t taddr = tmem + ((uint32_t)(32 * quad) << 16) + mb * ncols;
     const int out_w = kAbsorb ? kDC : kDH;
-    __nv_bfloat16* out = p.out + (int64_t)h * out_w + m0 + row;
+    __nv_bfloat16* out = p.out + (int64_t)h * out_w + m0 + 128 * mb + row;
     for (int c0 = 0; c0 < n; c0 += 16) {
       uint32_t r[16];
       tmem_ld16(taddr + c0, r);
@@ -151,12 +165,12 @@ __global__ void __launch_bounds__(128) proj_kernel(const __grid_constant__ Param
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, ncols);
+  if (warp == 0) tmem_dealloc(tmem, ncols * S::kMB);
 }
 
 size_t smem_bytes(bool absorb, int n_tile) {
-  const int chunks = absorb ? kDH / 64 : kDC / 64;
-  return (size_t)chunks * (128 * 64 * 2 + n_tile * 128) + 1024;
+  const int chunks = absorb ? kDH / 64 : kDC / 64, mbs = absorb ? Shape<true>::kMB : 1;
+  return (size_t)chunks * (mbs * 128 * 64 * 2 + n_tile * 128) + 1024;
 }
 
 // Batch rows per CTA: the whole batch up to 256 (one CTA per head and row block), else 256.
@@ -192,8 +206,8 @@ cudaError_t launch(int B, const void* act, int64_t ld_head, const void* w, void*
   const size_t smem = smem_bytes(kAbsorb, n_tile);
   cudaError_t e = cudaFuncSetAttribute(proj_kernel<kAbsorb>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(kAbsorb ? kDC / 128 : 1, kNH, (B + n_tile - 1) / n_tile);
-  return launch_pdl(proj_kernel<kAbsorb>, grid, dim3(128), smem, st, p);
+  const dim3 grid(kAbsorb ? kDC / 128 / Shape<kAbsorb>::kMB : 1, kNH, (B + n_tile - 1) / n_tile);
+  return launch_pdl(proj_kernel<kAbsorb>, grid, dim3(Shape<kAbsorb>::kThreads), smem, st, p);
 }
 
 }  // namespace proj_tc
