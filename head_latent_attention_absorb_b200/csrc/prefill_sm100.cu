@@ -277,12 +277,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
   AttnBars& bs = *reinterpret_cast<AttnBars*>(smem + AT_BAROFF);
   volatile int* abort_flag = &bs.abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // The query tiles of one (sequence, head) are consecutive blocks, the longest causal rows first:
-  // blocks that run together share that head's K/V tiles in L2 (read from HBM about once), and
-  // the short tiles of a head free their SMs early for the next head's long ones.
+  // A CTA takes a mirrored pair of query tiles of one (sequence, head), the longest causal rows
+  // first and then the shortest (n_qt + 1 key tiles together, the same for every pair), so the
+  // grid is balanced and half as large; the second tile's query load and first score MMAs overlap
+  // the first's tail.  The pairs of one (sequence, head) are consecutive blocks: blocks that run
+  // together share that head's K/V tiles in L2.
+  const int n_pairs = (p.n_qt + 1) / 2;
   const int idx = blockIdx.x;
-  const int qt = p.n_qt - 1 - idx % p.n_qt, h = (idx / p.n_qt) % p.H, b = idx / (p.n_qt * p.H);
-  const int n_kv = p.causal ? qt + 1 : p.n_qt;   // key tiles this query tile attends
+  const int pi = idx % n_pairs, h = (idx / n_pairs) % p.H, b = idx / (n_pairs * p.H);
+  const int n_items = (p.n_qt - 1 - pi != pi) ? 2 : 1;
+  auto item_qt = [&](int it) { return it == 0 ? p.n_qt - 1 - pi : pi; };
+  auto item_nkv = [&](int it) { return p.causal ? item_qt(it) + 1 : p.n_qt; };  // key tiles attended
 
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
@@ -316,34 +321,47 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
+    // K/V tiles of both query tiles go through one ring (global tile counter g); the second
+    // query tile's rows replace the first's in shared memory once the softmax warps have copied
+    // those into TMEM
     if (lane == 0) {
       griddep_wait();  // the expanded rows come from the preceding kernel
       const uint64_t pol = policy_evict_last();
       const uint32_t qb = smem_u32(&bs.q_tma);
-      mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
-      for (int sl = 0; sl < 3; ++sl)
-        tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * qt, b, pol);
       bool ok = true;
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const uint32_t st = j % AT_STAGES, ph = (j / AT_STAGES) & 1u;
-        if (!mbar_wait(smem_u32(&bs.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
+      int g = 0;
+      for (int it = 0; it < n_items && ok; ++it) {
+        const int qt = item_qt(it), n_kv = item_nkv(it);
+        if (it > 0 && !mbar_wait(smem_u32(&bs.q_full), (uint32_t)(it - 1) & 1u, abort_flag, kWaitLimitNs)) {
           fail();
           ok = false;
           break;
         }
-        const uint32_t dst = smem_u32(smem + AT_STAGE0 + st * AT_STAGE_BYTES);
-        const uint32_t bar = smem_u32(&bs.full[st]);
-        mbar_arrive_expect_tx(bar, AT_STAGE_BYTES);
-        tma_load_4d(dst, &p.tm_kv, bar, 0, h, AT_TILE * j, b, pol);                 // k_nope 0-63
-        tma_load_4d(dst + AT_SLAB, &p.tm_kv, bar, 64, h, AT_TILE * j, b, pol);      // k_nope 64-127
-        tma_load_3d(dst + 2 * AT_SLAB, &p.tm_kr, bar, 0, AT_TILE * j, b, pol);      // k_R
-        tma_load_4d(dst + 3 * AT_SLAB, &p.tm_kv, bar, 128, h, AT_TILE * j, b, pol); // v 0-63
-        tma_load_4d(dst + 4 * AT_SLAB, &p.tm_kv, bar, 192, h, AT_TILE * j, b, pol); // v 64-127
+        mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
+        for (int sl = 0; sl < 3; ++sl)
+          tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * qt, b, pol);
+        for (int j = 0; j < n_kv && ok; ++j, ++g) {
+          const uint32_t st = g % AT_STAGES, ph = (g / AT_STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&bs.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(smem + AT_STAGE0 + st * AT_STAGE_BYTES);
+          const uint32_t bar = smem_u32(&bs.full[st]);
+          mbar_arrive_expect_tx(bar, AT_STAGE_BYTES);
+          tma_load_4d(dst, &p.tm_kv, bar, 0, h, AT_TILE * j, b, pol);                 // k_nope 0-63
+          tma_load_4d(dst + AT_SLAB, &p.tm_kv, bar, 64, h, AT_TILE * j, b, pol);      // k_nope 64-127
+          tma_load_3d(dst + 2 * AT_SLAB, &p.tm_kr, bar, 0, AT_TILE * j, b, pol);      // k_R
+          tma_load_4d(dst + 3 * AT_SLAB, &p.tm_kv, bar, 128, h, AT_TILE * j, b, pol); // v 0-63
+          tma_load_4d(dst + 4 * AT_SLAB, &p.tm_kv, bar, 192, h, AT_TILE * j, b, pol); // v 64-127
+        }
       }
-      const int first = n_kv > AT_STAGES ? n_kv - AT_STAGES : 0;
-      for (int k = first; k < n_kv; ++k)
+      // drain: every load issued must have landed before the CTA may exit
+      const int first = g > AT_STAGES ? g - AT_STAGES : 0;
+      for (int k = first; k < g; ++k)
         mbar_wait(smem_u32(&bs.full[k % AT_STAGES]), (k / AT_STAGES) & 1u, abort_flag, kWaitLimitNs);
-      mbar_wait(qb, 0, abort_flag, kWaitLimitNs);
+      mbar_wait(qb, (uint32_t)(n_items - 1) & 1u, abort_flag, kWaitLimitNs);
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------------- MMA issuer
@@ -359,47 +377,50 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       }
       return ok;
     };
-    auto issue_pv = [&](int j) {
-      if (!wait_all(smem_u32(&bs.p_full[j & 1]), (j >> 1) & 1u)) return;
+    // O += P(g) V(g); `first`: the query tile's first key tile (O starts from it)
+    auto issue_pv = [&](int g, bool first) {
+      if (!wait_all(smem_u32(&bs.p_full[g & 1]), (g >> 1) & 1u)) return;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vb = smem_u32(smem + AT_STAGE0 + (j % AT_STAGES) * AT_STAGE_BYTES + 3 * AT_SLAB);
-        const uint32_t tP = tmem + AT_COL_S + 128 * (j & 1);
+        const uint32_t vb = smem_u32(smem + AT_STAGE0 + (g % AT_STAGES) * AT_STAGE_BYTES + 3 * AT_SLAB);
+        const uint32_t tP = tmem + AT_COL_S + 128 * (g & 1);
 #pragma unroll
         for (int k = 0; k < AT_TILE / 16; ++k)
           mma_ts(tmem + AT_COL_O, tP + 8 * k, smem_desc(vb + 2048 * k, AT_SLAB, 1024, kSwizzle128), idesc_pv,
-                 (j > 0 || k > 0) ? 1u : 0u);
-        mma_commit(smem_u32(&bs.empty[j % AT_STAGES]));
-        mma_commit(smem_u32(&bs.pv_done[j & 1]));
+                 (!first || k > 0) ? 1u : 0u);
+        mma_commit(smem_u32(&bs.empty[g % AT_STAGES]));
+        mma_commit(smem_u32(&bs.pv_done[g & 1]));
       }
       __syncwarp();
     };
-    if (wait_all(smem_u32(&bs.q_full), 0)) {
+    int g = 0;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int n_kv = item_nkv(it);
+      if (!wait_all(smem_u32(&bs.q_full), (uint32_t)it & 1u)) break;  // this query tile's rows in TMEM
       tc_fence_after();
-      for (int j = 0; j < n_kv && ok; ++j) {
-        // S(j) = Q K(j)^T into buffer j & 1, free once P.V(j - 2) has read the P it held
-        if (!wait_all(smem_u32(&bs.full[j % AT_STAGES]), (j / AT_STAGES) & 1u)) break;
-        if (j >= 2 && !wait_all(smem_u32(&bs.pv_done[j & 1]), ((j - 2) >> 1) & 1u)) break;
+      for (int j = 0; j < n_kv && ok; ++j, ++g) {
+        // S(g) = Q K(g)^T into buffer g & 1, free once P.V(g - 2) has read the P it held
+        if (!wait_all(smem_u32(&bs.full[g % AT_STAGES]), (g / AT_STAGES) & 1u)) break;
+        if (g >= 2 && !wait_all(smem_u32(&bs.pv_done[g & 1]), ((g - 2) >> 1) & 1u)) break;
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t kb = smem_u32(smem + AT_STAGE0 + (j % AT_STAGES) * AT_STAGE_BYTES);
-          const uint32_t tS = tmem + AT_COL_S + 128 * (j & 1);
+          const uint32_t kb = smem_u32(smem + AT_STAGE0 + (g % AT_STAGES) * AT_STAGE_BYTES);
+          const uint32_t tS = tmem + AT_COL_S + 128 * (g & 1);
 #pragma unroll
           for (int k = 0; k < 12; ++k)  // 8 K-steps of q_nope . k_nope, 4 of q_pe . k_R
             mma_ts(tS, tmem + AT_COL_Q + 8 * k, smem_desc(kb + (k >> 2) * AT_SLAB + 32 * (k & 3), 16, 1024, kSwizzle128),
                    idesc_qk, k > 0 ? 1u : 0u);
-          mma_commit(smem_u32(&bs.s_full[j & 1]));
+          mma_commit(smem_u32(&bs.s_full[g & 1]));
         }
         __syncwarp();
-        if (j >= 1) issue_pv(j - 1);  // P.V of the previous tile behind this tile's scores
+        if (j >= 1) issue_pv(g - 1, j == 1);  // P.V of the previous tile behind this tile's scores
       }
-      if (ok && n_kv > 0) issue_pv(n_kv - 1);
+      if (ok && n_kv > 0) issue_pv(g - 1, n_kv == 1);
     }
   } else {
     // ---------------------------------------------------------------- softmax (warps 2-5)
     const int quad = warp & 3;
     const int r = 32 * quad + lane;               // query row of this thread within the tile
-    const int q_pos = AT_TILE * qt + r;           // its position in the sequence
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
     const uint32_t tQ = tmem + lane_off + AT_COL_Q, tO = tmem + lane_off + AT_COL_O;
     bool ok = true;
@@ -412,8 +433,13 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       }
       return ok;
     };
-    // Q row -> TMEM (A operand): 192 features as 96 columns of bf16 pairs
-    if (wait_all(smem_u32(&bs.q_tma), 0)) {
+    int g = 0;
+    for (int it = 0; it < n_items && ok; ++it) {
+      const int qt = item_qt(it), n_kv = item_nkv(it);
+      const int q_pos = AT_TILE * qt + r;         // this row's position in the sequence
+      // Q row -> TMEM (A operand): 192 features as 96 columns of bf16 pairs.  For the second query
+      // tile every score MMA of the first is complete (its last scores were waited for).
+      if (!wait_all(smem_u32(&bs.q_tma), (uint32_t)it & 1u)) break;
       for (int sl = 0; sl < 3; ++sl) {
         const uint32_t row = smem_u32(smem + AT_QOFF + sl * AT_SLAB) + r * 128;
         uint32_t v[32];
@@ -428,90 +454,93 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bs.q_full));
-    }
-    float m_run = -INFINITY, l_run = 0.f;
-    for (int j = 0; j < n_kv && ok; ++j) {
-      if (!wait_all(smem_u32(&bs.s_full[j & 1]), (j >> 1) & 1u)) break;
-      tc_fence_after();
-      const uint32_t tS = tmem + lane_off + AT_COL_S + 128 * (j & 1);
-      const int key0 = AT_TILE * j;
-      // keys of this tile this row may attend: below the sequence length and (causal) <= q_pos
-      const int lim = p.causal ? min(p.S - 1, q_pos) : p.S - 1;
-      const int nvalid = lim - key0 + 1;  // keys 0 .. nvalid-1 of the tile are valid
-      // the whole score row in registers: four loads, one wait (the row is read from TMEM once)
-      uint32_t sv[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
-      tmem_ld_wait();
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int k = 0; k < 32; ++k)
-          if (32 * c + k < nvalid) mx = fmaxf(mx, __uint_as_float(sv[c][k]));
-      const float m_new = fmaxf(m_run, mx * p.scale_log2);
-      const bool need = m_new > m_run + 8.0f;  // true on the first tile (m_run = -inf)
-      if (j > 0 && __any_sync(0xffffffffu, need)) {
-        // O holds P.V of the earlier tiles relative to the old maximum: rescale it once the
-        // last of those products has landed
-        if (!wait_all(smem_u32(&bs.pv_done[(j - 1) & 1]), ((j - 1) >> 1) & 1u)) break;
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; j < n_kv && ok; ++j, ++g) {
+        if (!wait_all(smem_u32(&bs.s_full[g & 1]), (g >> 1) & 1u)) break;
         tc_fence_after();
-        const float corr = need ? ex2f_approx(m_run - m_new) : 1.f;
+        const uint32_t tS = tmem + lane_off + AT_COL_S + 128 * (g & 1);
+        const int key0 = AT_TILE * j;
+        // keys of this tile this row may attend: below the sequence length and (causal) <= q_pos
+        const int lim = p.causal ? min(p.S - 1, q_pos) : p.S - 1;
+        const int nvalid = lim - key0 + 1;  // keys 0 .. nvalid-1 of the tile are valid
+        // the whole score row in registers: four loads, one wait (the row is read from TMEM once)
+        uint32_t sv[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
+        tmem_ld_wait();
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int k = 0; k < 32; ++k)
+            if (32 * c + k < nvalid) mx = fmaxf(mx, __uint_as_float(sv[c][k]));
+        const float m_new = fmaxf(m_run, mx * p.scale_log2);
+        const bool need = m_new > m_run + 8.0f;  // true on the first tile (m_run = -inf)
+        if (j > 0 && __any_sync(0xffffffffu, need)) {
+          // O holds P.V of the earlier tiles relative to the old maximum: rescale it once the
+          // last of those products has landed
+          if (!wait_all(smem_u32(&bs.pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1u)) break;
+          tc_fence_after();
+          const float corr = need ? ex2f_approx(m_run - m_new) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t v[32];
+            tmem_ld32(tO + 32 * c, v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * corr);
+            tmem_st32(tO + 32 * c, v);
+          }
+        }
+        if (need) {
+          l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2f_approx(m_run - m_new);
+          m_run = m_new;
+        }
+        // P = 2^(s scale_log2 - m) in bf16, written over the scores it came from (chunk c of P takes
+        // columns [16c, 16c + 16); the whole row is already in registers)
+        float ls = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const int k0 = 32 * c + 2 * k;
+            const float p0 = k0 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k]), p.scale_log2, -m_run)) : 0.f;
+            const float p1 = k0 + 1 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k + 1]), p.scale_log2, -m_run)) : 0.f;
+            ls += p0 + p1;
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tS + 16 * c, pk);
+        }
+        l_run += ls;
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bs.p_full[g & 1]));
+      }
+      if (!ok) break;
+      // ---- epilogue of this query tile: O / l -> out (P.V of its last two tiles, older first)
+      if (n_kv >= 2 && !wait_all(smem_u32(&bs.pv_done[(g - 2) & 1]), ((g - 2) >> 1) & 1u)) break;
+      if (n_kv >= 1 && wait_all(smem_u32(&bs.pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1u)) {
+        tc_fence_after();
+        const float inv = 1.f / l_run;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
           tmem_ld32(tO + 32 * c, v);
           tmem_ld_wait();
+          if (q_pos < p.S) {
+            uint4* dst = reinterpret_cast<uint4*>(p.out + (((int64_t)b * p.S + q_pos) * p.H + h) * 128 + 32 * c);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) v[k] = __float_as_uint(__uint_as_float(v[k]) * corr);
-          tmem_st32(tO + 32 * c, v);
+            for (int w = 0; w < 4; ++w)
+              dst[w] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * w]) * inv, __uint_as_float(v[8 * w + 1]) * inv),
+                                  pack_bf16x2(__uint_as_float(v[8 * w + 2]) * inv, __uint_as_float(v[8 * w + 3]) * inv),
+                                  pack_bf16x2(__uint_as_float(v[8 * w + 4]) * inv, __uint_as_float(v[8 * w + 5]) * inv),
+                                  pack_bf16x2(__uint_as_float(v[8 * w + 6]) * inv, __uint_as_float(v[8 * w + 7]) * inv));
+          }
         }
-      }
-      if (need) {
-        l_run = (m_run == -INFINITY) ? 0.f : l_run * ex2f_approx(m_run - m_new);
-        m_run = m_new;
-      }
-      // P = 2^(s scale_log2 - m) in bf16, written over the scores it came from (chunk c of P takes
-      // columns [16c, 16c + 16); the whole row is already in registers)
-      float ls = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int k0 = 32 * c + 2 * k;
-          const float p0 = k0 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k]), p.scale_log2, -m_run)) : 0.f;
-          const float p1 = k0 + 1 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k + 1]), p.scale_log2, -m_run)) : 0.f;
-          ls += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16(tS + 16 * c, pk);
-      }
-      l_run += ls;
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bs.p_full[j & 1]));
-    }
-    // ---- epilogue: O / l -> out (P.V of the last two tiles, older first)
-    if (ok && n_kv >= 2) wait_all(smem_u32(&bs.pv_done[(n_kv - 2) & 1]), ((n_kv - 2) >> 1) & 1u);
-    if (ok && n_kv >= 1 && wait_all(smem_u32(&bs.pv_done[(n_kv - 1) & 1]), ((n_kv - 1) >> 1) & 1u)) {
-      tc_fence_after();
-      const float inv = 1.f / l_run;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + 32 * c, v);
-        tmem_ld_wait();
-        if (q_pos < p.S) {
-          uint4* dst = reinterpret_cast<uint4*>(p.out + (((int64_t)b * p.S + q_pos) * p.H + h) * 128 + 32 * c);
-#pragma unroll
-          for (int w = 0; w < 4; ++w)
-            dst[w] = make_uint4(pack_bf16x2(__uint_as_float(v[8 * w]) * inv, __uint_as_float(v[8 * w + 1]) * inv),
-                                pack_bf16x2(__uint_as_float(v[8 * w + 2]) * inv, __uint_as_float(v[8 * w + 3]) * inv),
-                                pack_bf16x2(__uint_as_float(v[8 * w + 4]) * inv, __uint_as_float(v[8 * w + 5]) * inv),
-                                pack_bf16x2(__uint_as_float(v[8 * w + 6]) * inv, __uint_as_float(v[8 * w + 7]) * inv));
-        }
+        // the next query tile's first P.V overwrites O: its P is written only after this read
+        tc_fence_before();
       }
     }
   }
@@ -601,7 +630,7 @@ cudaError_t attn_tc_launch(const PrefillArgs& a, cudaStream_t st) {
   const size_t smem = attn_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_kernel, dim3((unsigned)(p.n_qt * a.B * a.n_h)), dim3(AT_THREADS), smem, st, p);
+  return launch_pdl(attn_kernel, dim3((unsigned)((p.n_qt + 1) / 2 * a.B * a.n_h)), dim3(AT_THREADS), smem, st, p);
 }
 
 }  // namespace mla

@@ -289,6 +289,22 @@ def test_prefill_small_ragged(dev):
         check_close(out[b][:, list(range(0, 128, 7))], want, torch.bfloat16, f"prefill b={b}")
 
 
+@pytest.mark.parametrize("S,causal", [(100, True), (256, True), (600, True), (600, False), (384, False)])
+def test_prefill_query_tile_pairings(dev, S, causal):
+    # a CTA runs query tile n_qt-1-i and then tile i: one tile (S=100), an even tile count (256),
+    # an odd count whose middle tile runs alone (384, 600), causal and bidirectional
+    cfg = PREFILL.with_(B=2, n_max=S)
+    p = make_prefill_inputs(cfg)
+    out = api.mla_prefill_naive(cfg.dims, p["q"].cuda(), p["c_kv"].cuda(), p["k_r"].cuda(), p["w_kv_b"].cuda(),
+                                cfg.scale, causal=causal)
+    torch.cuda.synchronize()
+    heads = [0, 37, 127]
+    for b in range(cfg.B):
+        want = O.naive_prefill(p["q"][b], p["c_kv"][b], p["k_r"][b], p["w_kv_b"], cfg.scale, cfg.n_h, cfg.d_h,
+                               cfg.d_v, causal=causal, heads=heads)
+        check_close(out[b][:, heads], want, torch.bfloat16, f"prefill S={S} causal={causal} b={b}")
+
+
 # ------------------------------------------------------------------------------------------
 # Device-side error flag (no trap: the offending row is skipped)
 # ------------------------------------------------------------------------------------------
