@@ -238,7 +238,7 @@ static_assert(kBarOff + sizeof(Bars) + 1024 <= 232448, "dynamic shared memory ab
 // head, 128-query tile):
 //   * Q (128 x 192) is TMA-loaded once and copied into TMEM (A operand of S = Q K^T);
 //   * K tiles (128 keys: k_nope from the expanded rows, k_R shared by the heads) and V tiles stream
-//     through a 2-stage TMA ring;
+//     through two 2-stage TMA rings (a K stage is released by its score MMA, a V stage by its P.V);
 //   * S goes to one of two TMEM buffers; the softmax (4 warps, one query row per thread) takes the
 //     row maximum, then writes P = 2^(s - m) as bf16 over the same columns, and P.V reads it from
 //     TMEM (A operand) while the next S is computed into the other buffer;
@@ -248,10 +248,12 @@ static_assert(kBarOff + sizeof(Bars) + 1024 <= 232448, "dynamic shared memory ab
 constexpr int AT_TILE = 128;                      // queries per CTA, keys per tile
 constexpr int AT_SLAB = AT_TILE * 128;            // 128 rows x 64 bf16 (128-byte swizzle)
 constexpr int AT_QOFF = 0;                        // Q: 3 slabs (q_nope 0-63, 64-127, q_pe)
-constexpr int AT_STAGE0 = 3 * AT_SLAB;            // stage: K slabs (k_nope x2, k_R) + V slabs x2
-constexpr int AT_STAGE_BYTES = 5 * AT_SLAB;
-constexpr int AT_STAGES = 2;
-constexpr int AT_BAROFF = AT_STAGE0 + AT_STAGES * AT_STAGE_BYTES;
+constexpr int AT_STAGES = 2;                      // K and V rings of two stages each
+constexpr int AT_K0 = 3 * AT_SLAB;                // K stage: k_nope 0-63, 64-127, k_R
+constexpr int AT_KBYTES = 3 * AT_SLAB;
+constexpr int AT_V0 = AT_K0 + AT_STAGES * AT_KBYTES;  // V stage: v 0-63, 64-127
+constexpr int AT_VBYTES = 2 * AT_SLAB;
+constexpr int AT_BAROFF = AT_V0 + AT_STAGES * AT_VBYTES;
 constexpr int AT_THREADS = 192;                   // warp 0 loads, warp 1 MMAs, warps 2-5 softmax
 constexpr uint32_t AT_COL_Q = 0, AT_COL_S = 128, AT_COL_O = 384;  // Q 96 cols, S 2 x 128, O 128
 
@@ -266,7 +268,8 @@ struct AttnParams {
 };
 
 struct AttnBars {
-  uint64_t q_tma, q_full, full[AT_STAGES], empty[AT_STAGES], s_full[2], p_full[2], pv_done[2];
+  uint64_t q_tma, q_full, kfull[AT_STAGES], kempty[AT_STAGES], vfull[AT_STAGES], vempty[AT_STAGES];
+  uint64_t s_full[2], p_full[2], pv_done[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -294,8 +297,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     mbar_init(smem_u32(&bs.q_tma), 1);
     mbar_init(smem_u32(&bs.q_full), 4);
     for (int i = 0; i < 2; ++i) {
-      mbar_init(smem_u32(&bs.full[i]), 1);
-      mbar_init(smem_u32(&bs.empty[i]), 1);
+      mbar_init(smem_u32(&bs.kfull[i]), 1);
+      mbar_init(smem_u32(&bs.kempty[i]), 1);
+      mbar_init(smem_u32(&bs.vfull[i]), 1);
+      mbar_init(smem_u32(&bs.vempty[i]), 1);
       mbar_init(smem_u32(&bs.s_full[i]), 1);
       mbar_init(smem_u32(&bs.p_full[i]), 4);
       mbar_init(smem_u32(&bs.pv_done[i]), 1);
@@ -321,46 +326,71 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
 
   if (warp == 0) {
     // ---------------------------------------------------------------- TMA producer
-    // K/V tiles of both query tiles go through one ring (global tile counter g); the second
-    // query tile's rows replace the first's in shared memory once the softmax warps have copied
-    // those into TMEM
+    // Key tiles g = 0 .. G-1 of both query tiles in one sequence (global tile counter g).  K and V
+    // go through separate rings: a K stage is free once its score MMA has read it, a V stage once
+    // its P.V has, so the next key tile's load is not held behind the current softmax.  K runs one
+    // tile ahead of V in issue order.  The second query tile's rows replace the first's in shared
+    // memory once the softmax warps have copied those into TMEM.
     if (lane == 0) {
       griddep_wait();  // the expanded rows come from the preceding kernel
       const uint64_t pol = policy_evict_last();
       const uint32_t qb = smem_u32(&bs.q_tma);
+      const int n_kv0 = item_nkv(0);
+      const int G = n_kv0 + (n_items > 1 ? item_nkv(1) : 0);
+      auto key_row = [&](int g) { return AT_TILE * (g < n_kv0 ? g : g - n_kv0); };
       bool ok = true;
-      int g = 0;
-      for (int it = 0; it < n_items && ok; ++it) {
-        const int qt = item_qt(it), n_kv = item_nkv(it);
-        if (it > 0 && !mbar_wait(smem_u32(&bs.q_full), (uint32_t)(it - 1) & 1u, abort_flag, kWaitLimitNs)) {
-          fail();
-          ok = false;
-          break;
-        }
-        mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
-        for (int sl = 0; sl < 3; ++sl)
-          tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * qt, b, pol);
-        for (int j = 0; j < n_kv && ok; ++j, ++g) {
+      int nk = 0, nv = 0;  // K and V tiles issued
+      mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
+      for (int sl = 0; sl < 3; ++sl)
+        tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * item_qt(0), b, pol);
+      for (int s = 0; s <= G && ok; ++s) {
+        if (s < G) {
+          const int g = s;
+          if (g == n_kv0) {  // first key tile of the second query tile: its rows first
+            if (!mbar_wait(smem_u32(&bs.q_full), 0u, abort_flag, kWaitLimitNs)) {
+              fail();
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
+            for (int sl = 0; sl < 3; ++sl)
+              tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * item_qt(1), b, pol);
+          }
           const uint32_t st = g % AT_STAGES, ph = (g / AT_STAGES) & 1u;
-          if (!mbar_wait(smem_u32(&bs.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
+          if (!mbar_wait(smem_u32(&bs.kempty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
             fail();
             ok = false;
             break;
           }
-          const uint32_t dst = smem_u32(smem + AT_STAGE0 + st * AT_STAGE_BYTES);
-          const uint32_t bar = smem_u32(&bs.full[st]);
-          mbar_arrive_expect_tx(bar, AT_STAGE_BYTES);
-          tma_load_4d(dst, &p.tm_kv, bar, 0, h, AT_TILE * j, b, pol);                 // k_nope 0-63
-          tma_load_4d(dst + AT_SLAB, &p.tm_kv, bar, 64, h, AT_TILE * j, b, pol);      // k_nope 64-127
-          tma_load_3d(dst + 2 * AT_SLAB, &p.tm_kr, bar, 0, AT_TILE * j, b, pol);      // k_R
-          tma_load_4d(dst + 3 * AT_SLAB, &p.tm_kv, bar, 128, h, AT_TILE * j, b, pol); // v 0-63
-          tma_load_4d(dst + 4 * AT_SLAB, &p.tm_kv, bar, 192, h, AT_TILE * j, b, pol); // v 64-127
+          const uint32_t dst = smem_u32(smem + AT_K0 + st * AT_KBYTES);
+          const uint32_t bar = smem_u32(&bs.kfull[st]);
+          mbar_arrive_expect_tx(bar, AT_KBYTES);
+          tma_load_4d(dst, &p.tm_kv, bar, 0, h, key_row(g), b, pol);             // k_nope 0-63
+          tma_load_4d(dst + AT_SLAB, &p.tm_kv, bar, 64, h, key_row(g), b, pol);  // k_nope 64-127
+          tma_load_3d(dst + 2 * AT_SLAB, &p.tm_kr, bar, 0, key_row(g), b, pol);  // k_R
+          ++nk;
+        }
+        if (s >= 1) {
+          const int g = s - 1;
+          const uint32_t st = g % AT_STAGES, ph = (g / AT_STAGES) & 1u;
+          if (!mbar_wait(smem_u32(&bs.vempty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
+            fail();
+            ok = false;
+            break;
+          }
+          const uint32_t dst = smem_u32(smem + AT_V0 + st * AT_VBYTES);
+          const uint32_t bar = smem_u32(&bs.vfull[st]);
+          mbar_arrive_expect_tx(bar, AT_VBYTES);
+          tma_load_4d(dst, &p.tm_kv, bar, 128, h, key_row(g), b, pol);            // v 0-63
+          tma_load_4d(dst + AT_SLAB, &p.tm_kv, bar, 192, h, key_row(g), b, pol);  // v 64-127
+          ++nv;
         }
       }
       // drain: every load issued must have landed before the CTA may exit
-      const int first = g > AT_STAGES ? g - AT_STAGES : 0;
-      for (int k = first; k < g; ++k)
-        mbar_wait(smem_u32(&bs.full[k % AT_STAGES]), (k / AT_STAGES) & 1u, abort_flag, kWaitLimitNs);
+      for (int k = nk > AT_STAGES ? nk - AT_STAGES : 0; k < nk; ++k)
+        mbar_wait(smem_u32(&bs.kfull[k % AT_STAGES]), (k / AT_STAGES) & 1u, abort_flag, kWaitLimitNs);
+      for (int k = nv > AT_STAGES ? nv - AT_STAGES : 0; k < nv; ++k)
+        mbar_wait(smem_u32(&bs.vfull[k % AT_STAGES]), (k / AT_STAGES) & 1u, abort_flag, kWaitLimitNs);
       mbar_wait(qb, (uint32_t)(n_items - 1) & 1u, abort_flag, kWaitLimitNs);
     }
   } else if (warp == 1) {
@@ -380,15 +410,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     // O += P(g) V(g); `first`: the query tile's first key tile (O starts from it)
     auto issue_pv = [&](int g, bool first) {
       if (!wait_all(smem_u32(&bs.p_full[g & 1]), (g >> 1) & 1u)) return;
+      if (!wait_all(smem_u32(&bs.vfull[g % AT_STAGES]), (g / AT_STAGES) & 1u)) return;
       tc_fence_after();
       if (lane == 0) {
-        const uint32_t vb = smem_u32(smem + AT_STAGE0 + (g % AT_STAGES) * AT_STAGE_BYTES + 3 * AT_SLAB);
+        const uint32_t vb = smem_u32(smem + AT_V0 + (g % AT_STAGES) * AT_VBYTES);
         const uint32_t tP = tmem + AT_COL_S + 128 * (g & 1);
 #pragma unroll
         for (int k = 0; k < AT_TILE / 16; ++k)
           mma_ts(tmem + AT_COL_O, tP + 8 * k, smem_desc(vb + 2048 * k, AT_SLAB, 1024, kSwizzle128), idesc_pv,
                  (!first || k > 0) ? 1u : 0u);
-        mma_commit(smem_u32(&bs.empty[g % AT_STAGES]));
+        mma_commit(smem_u32(&bs.vempty[g % AT_STAGES]));
         mma_commit(smem_u32(&bs.pv_done[g & 1]));
       }
       __syncwarp();
@@ -400,17 +431,18 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       tc_fence_after();
       for (int j = 0; j < n_kv && ok; ++j, ++g) {
         // S(g) = Q K(g)^T into buffer g & 1, free once P.V(g - 2) has read the P it held
-        if (!wait_all(smem_u32(&bs.full[g % AT_STAGES]), (g / AT_STAGES) & 1u)) break;
+        if (!wait_all(smem_u32(&bs.kfull[g % AT_STAGES]), (g / AT_STAGES) & 1u)) break;
         if (g >= 2 && !wait_all(smem_u32(&bs.pv_done[g & 1]), ((g - 2) >> 1) & 1u)) break;
         tc_fence_after();
         if (lane == 0) {
-          const uint32_t kb = smem_u32(smem + AT_STAGE0 + (g % AT_STAGES) * AT_STAGE_BYTES);
+          const uint32_t kb = smem_u32(smem + AT_K0 + (g % AT_STAGES) * AT_KBYTES);
           const uint32_t tS = tmem + AT_COL_S + 128 * (g & 1);
 #pragma unroll
           for (int k = 0; k < 12; ++k)  // 8 K-steps of q_nope . k_nope, 4 of q_pe . k_R
             mma_ts(tS, tmem + AT_COL_Q + 8 * k, smem_desc(kb + (k >> 2) * AT_SLAB + 32 * (k & 3), 16, 1024, kSwizzle128),
                    idesc_qk, k > 0 ? 1u : 0u);
           mma_commit(smem_u32(&bs.s_full[g & 1]));
+          mma_commit(smem_u32(&bs.kempty[g % AT_STAGES]));
         }
         __syncwarp();
         if (j >= 1) issue_pv(g - 1, j == 1);  // P.V of the previous tile behind this tile's scores
@@ -468,12 +500,24 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
 #pragma unroll
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, sv[c]);
         tmem_ld_wait();
-        float mx = -INFINITY;
+        // masked keys (past the row's causal limit or the sequence end; only the diagonal and the
+        // last tile have any) become -inf: they leave the maximum alone and 2^-inf = 0
+        if (nvalid < AT_TILE) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+          for (int c = 0; c < 4; ++c)
 #pragma unroll
-          for (int k = 0; k < 32; ++k)
-            if (32 * c + k < nvalid) mx = fmaxf(mx, __uint_as_float(sv[c][k]));
+            for (int k = 0; k < 32; ++k)
+              sv[c][k] = 32 * c + k < nvalid ? sv[c][k] : 0xff800000u;
+        }
+        // row maximum and (below) row sum as eight and four independent chains, so the one warp
+        // on each sub-partition is not stalled on a 128-long dependency chain
+        float mxv[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mxv[k] = __uint_as_float(sv[0][k]);
+#pragma unroll
+        for (int i = 8; i < AT_TILE; ++i) mxv[i & 7] = fmaxf(mxv[i & 7], __uint_as_float(sv[i >> 5][i & 31]));
+        const float mx = fmaxf(fmaxf(fmaxf(mxv[0], mxv[1]), fmaxf(mxv[2], mxv[3])),
+                               fmaxf(fmaxf(mxv[4], mxv[5]), fmaxf(mxv[6], mxv[7])));
         const float m_new = fmaxf(m_run, mx * p.scale_log2);
         const bool need = m_new > m_run + 8.0f;  // true on the first tile (m_run = -inf)
         if (j > 0 && __any_sync(0xffffffffu, need)) {
@@ -498,21 +542,20 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
         }
         // P = 2^(s scale_log2 - m) in bf16, written over the scores it came from (chunk c of P takes
         // columns [16c, 16c + 16); the whole row is already in registers)
-        float ls = 0.f;
+        float lsv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const int k0 = 32 * c + 2 * k;
-            const float p0 = k0 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k]), p.scale_log2, -m_run)) : 0.f;
-            const float p1 = k0 + 1 < nvalid ? ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k + 1]), p.scale_log2, -m_run)) : 0.f;
-            ls += p0 + p1;
+            const float p0 = ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k]), p.scale_log2, -m_run));
+            const float p1 = ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k + 1]), p.scale_log2, -m_run));
+            lsv[k & 3] += p0 + p1;
             pk[k] = pack_bf16x2(p0, p1);
           }
           tmem_st16(tS + 16 * c, pk);
         }
-        l_run += ls;
+        l_run += (lsv[0] + lsv[1]) + (lsv[2] + lsv[3]);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
