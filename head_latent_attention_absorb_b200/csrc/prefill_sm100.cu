@@ -236,12 +236,12 @@ static_assert(kBarOff + sizeof(Bars) + 1024 <= 232448, "dynamic shared memory ab
 // Causal attention of the naive path ("Naive path": k = [k_nope; k_R broadcast], scores
 // q . k / sqrt(192), softmax over positions t <= s, output sum_t alpha_t v_t), per (sequence,
 // head, 128-query tile):
-//   * Q (128 x 192) is TMA-loaded once and copied into TMEM (A operand of S = Q K^T);
+//   * Q (128 x 192) is TMA-loaded once and read from shared memory by the score MMAs;
 //   * K tiles (128 keys: k_nope from the expanded rows, k_R shared by the heads) and V tiles stream
 //     through two 2-stage TMA rings (a K stage is released by its score MMA, a V stage by its P.V);
-//   * S goes to one of two TMEM buffers; the softmax (4 warps, one query row per thread) takes the
+//   * S goes to one of three TMEM buffers; the softmax (4 warps, one query row per thread) takes the
 //     row maximum, then writes P = 2^(s - m) as bf16 over the same columns, and P.V reads it from
-//     TMEM (A operand) while the next S is computed into the other buffer;
+//     TMEM (A operand) while the next S is computed into another buffer;
 //   * online softmax in base 2, the running maximum raised (and O rescaled) only when it grows by
 //     more than 8.
 // ------------------------------------------------------------------------------------------
@@ -255,7 +255,8 @@ constexpr int AT_V0 = AT_K0 + AT_STAGES * AT_KBYTES;  // V stage: v 0-63, 64-127
 constexpr int AT_VBYTES = 2 * AT_SLAB;
 constexpr int AT_BAROFF = AT_V0 + AT_STAGES * AT_VBYTES;
 constexpr int AT_THREADS = 192;                   // warp 0 loads, warp 1 MMAs, warps 2-5 softmax
-constexpr uint32_t AT_COL_Q = 0, AT_COL_S = 128, AT_COL_O = 384;  // Q 96 cols, S 2 x 128, O 128
+constexpr int AT_SBUF = 3;                        // score buffers in TMEM
+constexpr uint32_t AT_COL_S = 0, AT_COL_O = 384;  // S 3 x 128 columns, O 128
 
 struct AttnParams {
   CUtensorMap tm_q;   // 4-D (192, H, S, B) query rows, box (64, 1, 128, 1)
@@ -268,8 +269,8 @@ struct AttnParams {
 };
 
 struct AttnBars {
-  uint64_t q_tma, q_full, kfull[AT_STAGES], kempty[AT_STAGES], vfull[AT_STAGES], vempty[AT_STAGES];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t q_tma, q_free, kfull[AT_STAGES], kempty[AT_STAGES], vfull[AT_STAGES], vempty[AT_STAGES];
+  uint64_t s_full[AT_SBUF], p_full[AT_SBUF], pv_done[AT_SBUF];
   uint32_t tmem_base;
   int abort;
 };
@@ -295,12 +296,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bs.q_tma), 1);
-    mbar_init(smem_u32(&bs.q_full), 4);
-    for (int i = 0; i < 2; ++i) {
+    mbar_init(smem_u32(&bs.q_free), 1);
+    for (int i = 0; i < AT_STAGES; ++i) {
       mbar_init(smem_u32(&bs.kfull[i]), 1);
       mbar_init(smem_u32(&bs.kempty[i]), 1);
       mbar_init(smem_u32(&bs.vfull[i]), 1);
       mbar_init(smem_u32(&bs.vempty[i]), 1);
+    }
+    for (int i = 0; i < AT_SBUF; ++i) {
       mbar_init(smem_u32(&bs.s_full[i]), 1);
       mbar_init(smem_u32(&bs.p_full[i]), 4);
       mbar_init(smem_u32(&bs.pv_done[i]), 1);
@@ -330,7 +333,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     // go through separate rings: a K stage is free once its score MMA has read it, a V stage once
     // its P.V has, so the next key tile's load is not held behind the current softmax.  K runs one
     // tile ahead of V in issue order.  The second query tile's rows replace the first's in shared
-    // memory once the softmax warps have copied those into TMEM.
+    // memory once every score MMA of the first has completed.
     if (lane == 0) {
       griddep_wait();  // the expanded rows come from the preceding kernel
       const uint64_t pol = policy_evict_last();
@@ -346,16 +349,6 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       for (int s = 0; s <= G && ok; ++s) {
         if (s < G) {
           const int g = s;
-          if (g == n_kv0) {  // first key tile of the second query tile: its rows first
-            if (!mbar_wait(smem_u32(&bs.q_full), 0u, abort_flag, kWaitLimitNs)) {
-              fail();
-              ok = false;
-              break;
-            }
-            mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
-            for (int sl = 0; sl < 3; ++sl)
-              tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * item_qt(1), b, pol);
-          }
           const uint32_t st = g % AT_STAGES, ph = (g / AT_STAGES) & 1u;
           if (!mbar_wait(smem_u32(&bs.kempty[st]), ph ^ 1u, abort_flag, kWaitLimitNs)) {
             fail();
@@ -369,6 +362,16 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
           tma_load_4d(dst + AT_SLAB, &p.tm_kv, bar, 64, h, key_row(g), b, pol);  // k_nope 64-127
           tma_load_3d(dst + 2 * AT_SLAB, &p.tm_kr, bar, 0, key_row(g), b, pol);  // k_R
           ++nk;
+          if (g == n_kv0) {  // second query tile: its rows, once the first's score MMAs are done
+            if (!mbar_wait(smem_u32(&bs.q_free), 0u, abort_flag, kWaitLimitNs)) {
+              fail();
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
+            for (int sl = 0; sl < 3; ++sl)
+              tma_load_4d(smem_u32(smem + AT_QOFF + sl * AT_SLAB), &p.tm_q, qb, 64 * sl, h, AT_TILE * item_qt(1), b, pol);
+          }
         }
         if (s >= 1) {
           const int g = s - 1;
@@ -409,40 +412,44 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     };
     // O += P(g) V(g); `first`: the query tile's first key tile (O starts from it)
     auto issue_pv = [&](int g, bool first) {
-      if (!wait_all(smem_u32(&bs.p_full[g & 1]), (g >> 1) & 1u)) return;
+      if (!wait_all(smem_u32(&bs.p_full[g % AT_SBUF]), (g / AT_SBUF) & 1u)) return;
       if (!wait_all(smem_u32(&bs.vfull[g % AT_STAGES]), (g / AT_STAGES) & 1u)) return;
       tc_fence_after();
       if (lane == 0) {
         const uint32_t vb = smem_u32(smem + AT_V0 + (g % AT_STAGES) * AT_VBYTES);
-        const uint32_t tP = tmem + AT_COL_S + 128 * (g & 1);
+        const uint32_t tP = tmem + AT_COL_S + 128 * (g % AT_SBUF);
 #pragma unroll
         for (int k = 0; k < AT_TILE / 16; ++k)
           mma_ts(tmem + AT_COL_O, tP + 8 * k, smem_desc(vb + 2048 * k, AT_SLAB, 1024, kSwizzle128), idesc_pv,
                  (!first || k > 0) ? 1u : 0u);
         mma_commit(smem_u32(&bs.vempty[g % AT_STAGES]));
-        mma_commit(smem_u32(&bs.pv_done[g & 1]));
+        mma_commit(smem_u32(&bs.pv_done[g % AT_SBUF]));
       }
       __syncwarp();
     };
     int g = 0;
     for (int it = 0; it < n_items && ok; ++it) {
       const int n_kv = item_nkv(it);
-      if (!wait_all(smem_u32(&bs.q_full), (uint32_t)it & 1u)) break;  // this query tile's rows in TMEM
+      if (!wait_all(smem_u32(&bs.q_tma), (uint32_t)it & 1u)) break;  // this query tile's rows landed
       tc_fence_after();
       for (int j = 0; j < n_kv && ok; ++j, ++g) {
-        // S(g) = Q K(g)^T into buffer g & 1, free once P.V(g - 2) has read the P it held
+        // S(g) = Q K(g)^T into buffer g % 3, free once P.V(g - 3) has read the P it held: with three
+        // buffers that product was issued a whole tile earlier, so the score MMA does not wait
+        // for the tensor pipe to drain
         if (!wait_all(smem_u32(&bs.kfull[g % AT_STAGES]), (g / AT_STAGES) & 1u)) break;
-        if (g >= 2 && !wait_all(smem_u32(&bs.pv_done[g & 1]), ((g - 2) >> 1) & 1u)) break;
+        if (g >= AT_SBUF && !wait_all(smem_u32(&bs.pv_done[g % AT_SBUF]), ((g - AT_SBUF) / AT_SBUF) & 1u)) break;
         tc_fence_after();
         if (lane == 0) {
           const uint32_t kb = smem_u32(smem + AT_K0 + (g % AT_STAGES) * AT_KBYTES);
-          const uint32_t tS = tmem + AT_COL_S + 128 * (g & 1);
+          const uint32_t tS = tmem + AT_COL_S + 128 * (g % AT_SBUF);
+          const uint32_t qs = smem_u32(smem + AT_QOFF);
 #pragma unroll
           for (int k = 0; k < 12; ++k)  // 8 K-steps of q_nope . k_nope, 4 of q_pe . k_R
-            mma_ts(tS, tmem + AT_COL_Q + 8 * k, smem_desc(kb + (k >> 2) * AT_SLAB + 32 * (k & 3), 16, 1024, kSwizzle128),
-                   idesc_qk, k > 0 ? 1u : 0u);
-          mma_commit(smem_u32(&bs.s_full[g & 1]));
+            mma_ss(tS, smem_desc(qs + (k >> 2) * AT_SLAB + 32 * (k & 3), 16, 1024, kSwizzle128),
+                   smem_desc(kb + (k >> 2) * AT_SLAB + 32 * (k & 3), 16, 1024, kSwizzle128), idesc_qk, k > 0 ? 1u : 0u);
+          mma_commit(smem_u32(&bs.s_full[g % AT_SBUF]));
           mma_commit(smem_u32(&bs.kempty[g % AT_STAGES]));
+          if (j == n_kv - 1 && it + 1 < n_items) mma_commit(smem_u32(&bs.q_free));  // query rows reusable
         }
         __syncwarp();
         if (j >= 1) issue_pv(g - 1, j == 1);  // P.V of the previous tile behind this tile's scores
@@ -454,7 +461,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     const int quad = warp & 3;
     const int r = 32 * quad + lane;               // query row of this thread within the tile
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
-    const uint32_t tQ = tmem + lane_off + AT_COL_Q, tO = tmem + lane_off + AT_COL_O;
+    const uint32_t tO = tmem + lane_off + AT_COL_O;
     bool ok = true;
     auto wait_all = [&](uint32_t bar, uint32_t par) {
       if (!ok) return false;
@@ -469,28 +476,11 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     for (int it = 0; it < n_items && ok; ++it) {
       const int qt = item_qt(it), n_kv = item_nkv(it);
       const int q_pos = AT_TILE * qt + r;         // this row's position in the sequence
-      // Q row -> TMEM (A operand): 192 features as 96 columns of bf16 pairs.  For the second query
-      // tile every score MMA of the first is complete (its last scores were waited for).
-      if (!wait_all(smem_u32(&bs.q_tma), (uint32_t)it & 1u)) break;
-      for (int sl = 0; sl < 3; ++sl) {
-        const uint32_t row = smem_u32(smem + AT_QOFF + sl * AT_SLAB) + r * 128;
-        uint32_t v[32];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 u = ld_shared_v4_b32(row + ((c ^ (r & 7)) << 4));
-          v[4 * c] = u.x; v[4 * c + 1] = u.y; v[4 * c + 2] = u.z; v[4 * c + 3] = u.w;
-        }
-        tmem_st32(tQ + 32 * sl, v);
-      }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bs.q_full));
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; j < n_kv && ok; ++j, ++g) {
-        if (!wait_all(smem_u32(&bs.s_full[g & 1]), (g >> 1) & 1u)) break;
+        if (!wait_all(smem_u32(&bs.s_full[g % AT_SBUF]), (g / AT_SBUF) & 1u)) break;
         tc_fence_after();
-        const uint32_t tS = tmem + lane_off + AT_COL_S + 128 * (g & 1);
+        const uint32_t tS = tmem + lane_off + AT_COL_S + 128 * (g % AT_SBUF);
         const int key0 = AT_TILE * j;
         // keys of this tile this row may attend: below the sequence length and (causal) <= q_pos
         const int lim = p.causal ? min(p.S - 1, q_pos) : p.S - 1;
@@ -523,7 +513,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
         if (j > 0 && __any_sync(0xffffffffu, need)) {
           // O holds P.V of the earlier tiles relative to the old maximum: rescale it once the
           // last of those products has landed
-          if (!wait_all(smem_u32(&bs.pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1u)) break;
+          if (!wait_all(smem_u32(&bs.pv_done[(g - 1) % AT_SBUF]), ((g - 1) / AT_SBUF) & 1u)) break;
           tc_fence_after();
           const float corr = need ? ex2f_approx(m_run - m_new) : 1.f;
 #pragma unroll 1
@@ -559,12 +549,12 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&bs.p_full[g & 1]));
+        if (lane == 0) mbar_arrive(smem_u32(&bs.p_full[g % AT_SBUF]));
       }
       if (!ok) break;
-      // ---- epilogue of this query tile: O / l -> out (P.V of its last two tiles, older first)
-      if (n_kv >= 2 && !wait_all(smem_u32(&bs.pv_done[(g - 2) & 1]), ((g - 2) >> 1) & 1u)) break;
-      if (n_kv >= 1 && wait_all(smem_u32(&bs.pv_done[(g - 1) & 1]), ((g - 1) >> 1) & 1u)) {
+      // ---- epilogue of this query tile: O / l -> out, once its last P.V (and so every earlier one)
+      // has completed
+      if (n_kv >= 1 && wait_all(smem_u32(&bs.pv_done[(g - 1) % AT_SBUF]), ((g - 1) / AT_SBUF) & 1u)) {
         tc_fence_after();
         const float inv = 1.f / l_run;
 #pragma unroll 1
