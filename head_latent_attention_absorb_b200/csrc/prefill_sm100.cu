@@ -275,6 +275,20 @@ struct AttnBars {
   int abort;
 };
 
+// Non-blocking check of an mbarrier phase: when the phase has already completed it answers
+// without the suspend-and-wake of try_wait.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -403,7 +417,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     bool ok = true;
     auto wait_all = [&](uint32_t bar, uint32_t par) {
       if (!ok) return false;
-      const bool mine = mbar_wait(bar, par, abort_flag, kWaitLimitNs);
+      const bool mine = mbar_test_wait(bar, par) || mbar_wait(bar, par, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, mine)) {
         if (lane == 0) fail();
         ok = false;
@@ -465,7 +479,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
     bool ok = true;
     auto wait_all = [&](uint32_t bar, uint32_t par) {
       if (!ok) return false;
-      const bool mine = mbar_wait(bar, par, abort_flag, kWaitLimitNs);
+      const bool mine = mbar_test_wait(bar, par) || mbar_wait(bar, par, abort_flag, kWaitLimitNs);
       if (!__all_sync(0xffffffffu, mine)) {
         if (lane == 0) fail();
         ok = false;
