@@ -165,10 +165,11 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill")):
+def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append")):
     """The other workloads of the hot path, each timed on its own with CUDA events (L2 flushed
-    before every launch): the ragged long-context decode, the V3.2 top-k decode and the naive causal
-    prefill.  Reported beside the headline line; algorithmic bytes / FLOPs as for the headline."""
+    before every launch): the ragged long-context decode, the V3.2 top-k decode, the naive causal
+    prefill and the cache append of one new token per sequence in front of the decode.  Reported
+    beside the headline line; algorithmic bytes / FLOPs as for the headline."""
     from head_latent_attention_absorb_b200 import api
     from head_latent_attention_absorb_b200.configs import PREFILL, RAGGED_LONG, SPARSE_V32
     from head_latent_attention_absorb_b200.inputs import make_prefill_inputs
@@ -209,6 +210,25 @@ def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill")):
                          "keys": keys, "algorithmic_bytes": nbytes, "achieved_GBs": gbs,
                          "hbm_frac": gbs / peaks["hbm_gbs"], "tflops": flops / (ms * 1e-3) / 1e12}
         del x, cache, c_kv, k_r, ws
+        torch.cuda.empty_cache()
+    if "append" in which:
+        # one new token for each of the decode workload's 32 sequences, written into its cache
+        cfg = V3_DECODE
+        rng = np.random.default_rng(cfg.seed + 100)
+        kv_a = torch.from_numpy(rng.standard_normal((cfg.B, cfg.d_c + cfg.d_r), dtype=np.float32)).to(
+            torch.bfloat16).to(dev)
+        gain = torch.ones((cfg.d_c,), dtype=torch.float32, device=dev)
+        cache = torch.zeros((cfg.B, cfg.n_max, cfg.d_c + cfg.d_r), dtype=torch.bfloat16, device=dev)
+        pos = torch.full((cfg.B,), cfg.n_max - 1, dtype=torch.int32, device=dev)
+        ms = timed(lambda: api.mla_cache_append(cfg.dims, kv_a, pos, cache[..., :cfg.d_c], cache[..., cfg.d_c:],
+                                                gain, stream=stream))
+        row = (cfg.d_c + cfg.d_r) * 2
+        nbytes = cfg.B * (2 * row + 4) + cfg.d_c * 4
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        out["append_b32"] = {"call": "mla_cache_append", "ms": ms, "tokens_per_s": cfg.B / (ms * 1e-3),
+                             "algorithmic_bytes": nbytes, "achieved_GBs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                             "note": "a few KB per call: bound by launch latency, not by HBM"}
+        del cache
         torch.cuda.empty_cache()
     if "prefill" not in which:
         return out
@@ -391,7 +411,7 @@ def main():
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the timings of the ragged, top-k and prefill workloads")
-    ap.add_argument("--only", choices=["ragged", "sparse", "prefill"],
+    ap.add_argument("--only", choices=["ragged", "sparse", "prefill", "append"],
                     help="time only this secondary workload (--steps launches after 3 warm-up ones) and print "
                          "its entry; a small command for profilers, not a bench line")
     args = ap.parse_args()

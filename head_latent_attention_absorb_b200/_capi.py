@@ -47,6 +47,8 @@ SIGNATURES = {
     "mla_prefill_workspace_size": (c_sz, [MLADims, c_i32, c_i32, c_i32]),
     "mla_prefill_naive": (c_i32, [MLADims, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp,
                                   c_f32, c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "mla_cache_append": (c_i32, [MLADims, c_i32, c_i32, c_vp, c_i64, c_vp, c_f32, c_f32, c_vp, c_i32,
+                                 c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp]),
     "mla_clear_device_error": (c_i32, [c_vp, c_vp]),
     "mla_get_device_error": (c_i32, [c_vp, c_i32p]),
 }

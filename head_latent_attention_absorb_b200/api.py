@@ -176,6 +176,30 @@ def mla_prefill_naive(dims, q: torch.Tensor, c_kv: torch.Tensor, k_r: torch.Tens
     return out
 
 
+def mla_cache_append(dims, kv_a: torch.Tensor, positions: torch.Tensor, c_kv: torch.Tensor, k_r: torch.Tensor,
+                     gain: Optional[torch.Tensor] = None, eps: float = 1e-6, rope_base: float = 10000.0,
+                     dev_err: Optional[torch.Tensor] = None, stream=None) -> None:
+    """Write each sequence's new token into the caches in place: RMSNorm(kv_a[b, :d_c]) * gain into
+    c_kv[b, positions[b]] and the rotary key kv_a[b, d_c:] rotated by positions[b] into
+    k_r[b, positions[b]].  kv_a [B, d_c + d_r] (rows may be strided); positions int32 [B];
+    c_kv [B, n_max, d_c] and k_r [B, n_max, d_r] may be views of one packed cache; gain fp32 [d_c]."""
+    d = _dims(dims)
+    B, n_max = c_kv.shape[0], c_kv.shape[1]
+    _rows(kv_a, "kv_a")
+    _rows(c_kv, "c_kv")
+    _rows(k_r, "k_r")
+    if kv_a.dim() != 2 or kv_a.shape[0] != B:
+        raise ValueError("kv_a must be [B, d_c + d_r]")
+    if positions.dtype != torch.int32 or not positions.is_contiguous():
+        raise TypeError("positions must be a contiguous int32 tensor")
+    if gain is not None and (gain.dtype != torch.float32 or not gain.is_contiguous()):
+        raise TypeError("gain must be a contiguous float32 tensor")
+    check(lib().mla_cache_append(d, _dt(kv_a), B, _ptr(kv_a), kv_a.stride(0), _ptr(gain), float(eps),
+                                 float(rope_base), _ptr(positions), n_max,
+                                 _ptr(c_kv), c_kv.stride(0), c_kv.stride(1), _ptr(k_r), k_r.stride(0),
+                                 k_r.stride(1), _ptr(dev_err), _stream(stream)), "mla_cache_append")
+
+
 def mla_clear_device_error(dev_err: torch.Tensor, stream=None) -> None:
     check(lib().mla_clear_device_error(_ptr(dev_err), _stream(stream)), "mla_clear_device_error")
 

@@ -62,6 +62,18 @@ struct PrefillArgs {
   void* kv;  // expanded [B, S, n_h, d_h + d_v] in the input dtype
 };
 
+// Validated arguments of one cache append (one new token per sequence).
+struct AppendArgs {
+  int d_c, d_r, B, n_max;
+  const void* kv_a; int64_t lda;  // [B, d_c + d_r] rows: latent first, rotary key last
+  const float* gain;              // [d_c] RMSNorm gain, or nullptr for ones
+  float eps, rope_base;
+  const int32_t* positions;       // [B] cache row (= position) of each new token
+  void* c_kv; int64_t ckv_b, ckv_r;
+  void* k_r;  int64_t kr_b, kr_r;
+  int32_t* err;
+};
+
 // Launch with programmatic stream serialization: the kernel may start while the preceding kernel
 // in the stream is still running, and synchronises with it through griddepcontrol.wait before it
 // touches that kernel's data (every kernel of this library does).

@@ -23,6 +23,10 @@ cudaError_t prefill_simt_launch(const PrefillArgs& a, cudaStream_t st);
 
 int decode_simt_splits(int B, int n_keys_cap);
 
+// ---- cache append (any dimensions; float or __nv_bfloat16) ---------------------------------
+template <typename T>
+cudaError_t cache_append_launch(const AppendArgs& a, cudaStream_t st);
+
 // ---- tcgen05 kernels (bf16, DeepSeek-V3 dimensions) ------------------------------------------
 size_t decode_tc_workspace(int B);
 cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st);

@@ -268,6 +268,41 @@ mla_status mla_prefill_naive(mla_dims dims, mla_dtype dtype, int32_t B, int32_t 
   return cuda_status(e, "mla_prefill_naive launch");
 }
 
+mla_status mla_cache_append(mla_dims dims, mla_dtype dtype, int32_t B, const void* kv_a, int64_t lda,
+                            const float* gain, float eps, float rope_base, const int32_t* positions, int32_t n_max,
+                            void* c_kv, int64_t ckv_bstride, int64_t ckv_rstride, void* k_r, int64_t kr_bstride,
+                            int64_t kr_rstride, int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0 || n_max <= 0) return fail(MLA_ERR_INVALID_ARG, "B and n_max must be positive");
+  if (!kv_a || !positions || !c_kv || !k_r) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (dims.d_r % 2 != 0) return fail(MLA_ERR_INVALID_ARG, "d_r must be even (rotary pairs)");
+  if (lda < (int64_t)dims.d_c + dims.d_r) return fail(MLA_ERR_INVALID_ARG, "lda smaller than d_c + d_r");
+  if (ckv_rstride < dims.d_c || kr_rstride < dims.d_r) return fail(MLA_ERR_INVALID_ARG, "row stride too small");
+  if (ckv_bstride < (int64_t)n_max * ckv_rstride || kr_bstride < (int64_t)n_max * kr_rstride)
+    return fail(MLA_ERR_INVALID_ARG, "batch stride smaller than n_max rows");
+  if (!(eps >= 0.f) || !(eps < 1e30f)) return fail(MLA_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (!(rope_base > 0.f) || !(rope_base < 1e30f)) return fail(MLA_ERR_INVALID_ARG, "rope_base must be finite and > 0");
+  MLA_TRY(check_bf16_ptr(dtype, kv_a, "kv_a"));
+  MLA_TRY(check_bf16_ptr(dtype, c_kv, "c_kv"));
+  MLA_TRY(check_bf16_ptr(dtype, k_r, "k_r"));
+  MLA_TRY(check_bf16_stride(dtype, lda, "lda"));
+  MLA_TRY(check_bf16_stride(dtype, ckv_rstride, "ckv_rstride"));
+  MLA_TRY(check_bf16_stride(dtype, kr_rstride, "kr_rstride"));
+  MLA_TRY(check_bf16_stride(dtype, ckv_bstride, "ckv_bstride"));
+  MLA_TRY(check_bf16_stride(dtype, kr_bstride, "kr_bstride"));
+  mla::AppendArgs a;
+  a.d_c = dims.d_c; a.d_r = dims.d_r; a.B = B; a.n_max = n_max;
+  a.kv_a = kv_a; a.lda = lda; a.gain = gain; a.eps = eps; a.rope_base = rope_base; a.positions = positions;
+  a.c_kv = c_kv; a.ckv_b = ckv_bstride; a.ckv_r = ckv_rstride;
+  a.k_r = k_r; a.kr_b = kr_bstride; a.kr_r = kr_rstride;
+  a.err = dev_err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = dtype == MLA_BF16 ? mla::cache_append_launch<__nv_bfloat16>(a, st)
+                                          : mla::cache_append_launch<float>(a, st);
+  return cuda_status(e, "mla_cache_append launch");
+}
+
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream) {
   g_msg[0] = 0;
   if (!dev_err) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");

@@ -10,6 +10,9 @@
  *   mla_prefill_naive  wkv_b expansion, k = [k_nope; k^R], causal attention
  *                                                                    ("Value up-projection", prefill excerpt;
  *                                                                     "KV Reconstruction", "Naive path")
+ *   mla_cache_append   the new token's latent (RMSNorm) and rotary key (RoPE) into the caches
+ *                                                                    ("Key-value down-projection", mla-kv
+ *                                                                     excerpt; "Key-value latent RMSNorm")
  *
  * Conventions shared by every call
  * --------------------------------
@@ -47,7 +50,8 @@ typedef enum {
   MLA_ERR_INVALID_ARG = 1,  /* NULL pointer, non-positive size, misaligned pointer or stride  */
   MLA_ERR_UNSUPPORTED = 2,  /* dimensions / dtype combination without a kernel               */
   MLA_ERR_CUDA = 3,         /* a CUDA runtime call failed (see mla_last_error_message)       */
-  MLA_ERR_INDEX = 4,        /* device flag: a top-k index outside [0, length)                */
+  MLA_ERR_INDEX = 4,        /* device flag: a top-k index outside [0, length), or an append
+                               position outside [0, n_max)                                    */
   MLA_ERR_TIMEOUT = 5,      /* device flag: a bounded wait inside a kernel ran out           */
   MLA_ERR_WORKSPACE = 6,    /* workspace NULL or smaller than the matching *_workspace_size  */
   MLA_ERR_LENGTH = 7        /* device flag: a sequence length outside [1, n_max]             */
@@ -190,6 +194,31 @@ mla_status mla_prefill_naive(mla_dims dims, mla_dtype dtype, int32_t B, int32_t 
                              const void* k_r, int64_t kr_rstride, const void* w_kv_b,
                              float scale, int32_t causal, void* out,
                              void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * mla_cache_append - write one new token per sequence into the latent and rotary caches, the
+ * step that precedes the decode ("Key-value down-projection", mla-kv excerpt: the joint
+ * down-projection is split into the latent and the rotary key, the latent goes through kv_norm
+ * and the key through the rotary embedding; "Key-value latent RMSNorm": fp32, one gain per
+ * feature, eps inside the square root).  The pages do not show the cache write or the rotary
+ * convention; the reading taken here is the decode's: row t of both caches holds position t.
+ *   kv_a       new rows, element (b, j) at kv_a[b*lda + j]; j < d_c latent, d_c <= j < d_c+d_r rotary
+ *   gain       DEVICE fp32 [d_c] RMSNorm gain, or NULL for ones
+ *   positions  DEVICE int32 [B]: position p_b of each new token = the cache row it is written to
+ *   c_kv       c_kv[b*ckv_bstride + p_b*ckv_rstride + c] = gain[c] * x_c / sqrt(mean_c(x_c^2) + eps),
+ *              x = kv_a[b, 0:d_c] in fp32
+ *   k_r        pair i of k_r[b*kr_bstride + p_b*kr_rstride + :] = (y[2i] + j y[2i+1]) exp(j p_b base^(-2i/d_r)),
+ *              y = kv_a[b, d_c:d_c+d_r]: interleaved pairs, base = rope_base (10000 in DeepSeek-V3)
+ *   Every other cache row is left as it was.  d_r must be even; eps >= 0; rope_base > 0.
+ *   Device flag: a position outside [0, n_max) sets MLA_ERR_INDEX and that sequence writes nothing.
+ * Asynchronous on `stream`.
+ */
+mla_status mla_cache_append(mla_dims dims, mla_dtype dtype, int32_t B,
+                            const void* kv_a, int64_t lda, const float* gain, float eps, float rope_base,
+                            const int32_t* positions, int32_t n_max,
+                            void* c_kv, int64_t ckv_bstride, int64_t ckv_rstride,
+                            void* k_r, int64_t kr_bstride, int64_t kr_rstride,
+                            int32_t* dev_err, void* stream);
 
 /* Zero the device flag (asynchronous on `stream`). */
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream);

@@ -8,13 +8,14 @@ binding) never does, and shares no code with it.
 Pinned against what the pages and the mathematics fix (see ``tests/test_oracle_pins.py``):
 the absorb/naive identity, closed forms (one cached row, zero query, two keys),
 library special cases (``scaled_dot_product_attention`` in fp64), brute-force
-top-k masking, the page's parameter counts and cache-size formulas, and planted
-mistakes that must be caught.  Every function here has at least one such pin.
+top-k masking, the page's parameter counts and cache-size formulas, the RMSNorm and
+rotation invariants of the cache append, and planted mistakes that must be caught.  Every function here has at least one such pin.
 """
 
 from .mla_oracle import (  # noqa: F401
     absorb_q,
     absorbed_decode,
+    cache_append,
     index_mask,
     latent_attention,
     mha_cache_bytes,
@@ -22,6 +23,8 @@ from .mla_oracle import (  # noqa: F401
     naive_decode,
     naive_prefill,
     out_up,
+    rms_norm,
+    rope_interleaved,
     softmax,
     softmax_scale,
     split_wkv_b,

@@ -27,11 +27,17 @@ Sources (page title, then section / equation):
 * "Value up-projection", "Parameters": 8,388,608 parameters per value up-projection.
 * "DeepSeek V3" (rainlin-net), "Decoupled RoPE": MLA cache = B N (d_c + d_R) s bytes,
   against 2 B N h_q d_h s for standard MHA.
+* "DeepSeek-V3.2-Exp - Key-value down-projection", the mla-kv excerpt: the joint down-projection
+  is split into the latent (kv_lora_rank) and the rotary key (qk_rope_head_dim); the latent goes
+  through kv_norm, the key through the rotary embedding.  "Key-value latent RMSNorm": float32,
+  x rsqrt(mean(x^2) + eps), then one gain per feature.
 
 Readings where the pages are silent (each listed in the design notes):
 * Mask semantics: a scatter of 0 into a -inf row is a set, so a repeated index counts once.
 * Causal prefill: query position s attends keys t <= s.
 * One query token per sequence in decode; the query is the last cached position.
+* Rotary embedding: interleaved pairs rotated by pos base^(-2i/d) (the rotation is not shown);
+  the new token's rows are written at cache row = its position.
 """
 
 from __future__ import annotations
@@ -238,3 +244,40 @@ def absorbed_decode(q_nope, q_pe, c_kv, k_r, w_kv_b, scale: float, d_v: int, top
 def softmax_scale(d_h: int, d_r: int) -> float:
     """qk_head_dim^-0.5 with qk_head_dim = d_h + d_r ("Key-value latent", MLA-init excerpt)."""
     return 1.0 / math.sqrt(d_h + d_r)
+
+
+# ----------------------------------------------------------------------------------------
+# The step before the path: the new token's latent and rotary key into the caches
+# ----------------------------------------------------------------------------------------
+
+def rms_norm(x, gain=None, eps: float = 1e-6) -> np.ndarray:
+    """"Key-value latent RMSNorm": each row divided by the square root of (the mean of its
+    squares + eps), then multiplied by one gain per feature (ones when ``gain`` is None)."""
+    x = _f64(x)
+    y = x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    return y if gain is None else y * _f64(gain)
+
+
+def rope_interleaved(y, positions, base: float = 10000.0) -> np.ndarray:
+    """Rotary embedding of the shared key ("Key-value down-projection", mla-kv excerpt; the
+    rotation itself is not shown on the pages).  Reading taken: pair i = (y[2i], y[2i+1]) is the
+    complex number y[2i] + j y[2i+1], multiplied by exp(j pos base^(-2i/d)), pos = the row's
+    position.  ``y`` [rows, d], ``positions`` [rows]."""
+    y = _f64(y)
+    d = y.shape[-1]
+    pos = np.asarray(positions, dtype=np.float64)
+    freq = base ** (-np.arange(0, d, 2, dtype=np.float64) / d)       # [d/2]
+    z = (y[..., 0::2] + 1j * y[..., 1::2]) * np.exp(1j * pos[:, None] * freq[None, :])
+    out = np.empty_like(y)
+    out[..., 0::2], out[..., 1::2] = z.real, z.imag
+    return out
+
+
+def cache_append(kv_a, positions, d_c: int, d_r: int, gain=None, eps: float = 1e-6,
+                 base: float = 10000.0):
+    """The new token's cache rows ("Key-value down-projection", mla-kv excerpt): split the joint
+    down-projection row into the d_c latent and the d_r rotary key, RMSNorm the latent, rotate
+    the key.  Returns (latent rows [B, d_c], rotary rows [B, d_r]); row b belongs at cache row
+    positions[b] (the decode reads row t as position t)."""
+    x = _f64(kv_a)
+    return rms_norm(x[:, :d_c], gain, eps), rope_interleaved(x[:, d_c:d_c + d_r], positions, base)

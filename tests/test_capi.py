@@ -91,6 +91,25 @@ def test_host_validation_codes(L):
     # prefill
     assert L.mla_prefill_naive(DS, bf, 1, 16, FAKE, FAKE, 576, FAKE, 576, FAKE, 0.07, 1, FAKE, None, 0, None) == 6
     assert L.mla_prefill_naive(DS, bf, 1, 0, FAKE, FAKE, 576, FAKE, 576, FAKE, 0.07, 1, FAKE, FAKE, 1 << 30, None) == 1
+    # cache append
+    def app(**kw):
+        a = dict(dims=DS, dt=bf, B=2, kv=FAKE, lda=576, gain=None, eps=1e-6, base=10000.0, pos=FAKE, n_max=64,
+                 ckv=FAKE, cb=64 * 576, cr=576, kr=FAKE, kb=64 * 576, krr=576, err=None)
+        a.update(kw)
+        return L.mla_cache_append(*a.values(), None)
+
+    assert app(pos=None) == 1
+    assert app(B=0) == 1
+    assert app(lda=500) == 1                # narrower than d_c + d_r
+    assert app(cr=577) == 1                 # not a multiple of 8 elements
+    assert app(cb=63 * 576) == 1            # batch stride below n_max rows
+    assert app(eps=-1.0) == 1
+    assert app(base=0.0) == 1
+    assert app(kv=FAKE + 2) == 1            # misaligned bf16 row
+    assert L.mla_cache_append(_capi.MLADims(4, 64, 15, 32, 32), f32, 1, FAKE, 79, None, 1e-6, 1e4, FAKE, 8,
+                              FAKE, 8 * 64, 64, FAKE, 8 * 15, 15, None, None) == 1   # odd rotary width
+    assert L.mla_cache_append(tiny, bf, 1, FAKE, 80, None, 1e-6, 1e4, FAKE, 8,
+                              FAKE, 8 * 64, 64, FAKE, 8 * 16, 16, None, None) == 2   # bf16 outside DeepSeek dims
     assert L.mla_clear_device_error(None, None) == 1
     out = ctypes.c_int32(0)
     assert L.mla_get_device_error(None, ctypes.byref(out)) == 1
