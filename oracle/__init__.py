@@ -16,10 +16,12 @@ from .mla_oracle import (  # noqa: F401
     absorb_q,
     absorbed_decode,
     cache_append,
+    fp8_block_scale_shape,
     index_mask,
     latent_attention,
     mha_cache_bytes,
     mla_cache_bytes,
+    multi_token_decode,
     naive_decode,
     naive_prefill,
     out_up,
@@ -29,4 +31,5 @@ from .mla_oracle import (  # noqa: F401
     softmax_scale,
     split_wkv_b,
     value_up_params,
+    weight_dequant,
 )

@@ -167,7 +167,7 @@ def naive_decode(q_nope, q_pe, c_kv, k_r, w_kv_b, scale: float, topk=None, heads
 
 
 def naive_prefill(q, c_kv, k_r, w_kv_b, scale: float, n_h: int, d_h: int, d_v: int,
-                  causal: bool = True, rows=None, heads=None):
+                  causal: bool = True, rows=None, heads=None, topk=None):
     """Naive MLA prefill for ONE sequence ("Value up-projection", MHA-prefill excerpt).
 
     q [S, n_h, d_h + d_r] (content part first, rotary part last), c_kv [S, d_c], k_r [S, d_r].
@@ -176,6 +176,10 @@ def naive_prefill(q, c_kv, k_r, w_kv_b, scale: float, n_h: int, d_h: int, d_v: i
 
     Steps: kv = W_kv_b c (viewed [S, n_h, d_h + d_v]) -> k_nope, v; k = [k_nope; k_pe broadcast];
     scores = q . k * scale; causal additive mask (t <= s kept); softmax over t; out = sum alpha v.
+    Sparse variant (the V3.2 MHA-prefill excerpt): ``topk`` [S, k] holds each query row's selected
+    positions; a -inf row with 0 scattered at them is added to the causal mask and then to the
+    scores, so row s attends its selected positions t <= s (a set: repeats count once).  Every
+    row's set must hold at least one t <= s.
     Returns out [len(rows), len(heads), d_v].
     """
     q, c_kv, k_r = map(_f64, (q, c_kv, k_r))
@@ -188,10 +192,14 @@ def naive_prefill(q, c_kv, k_r, w_kv_b, scale: float, n_h: int, d_h: int, d_v: i
     k = np.concatenate([k_nope, np.broadcast_to(k_r[:, None, :], (S, len(hs), k_r.shape[1]))], axis=-1)
     qs = q[rs][:, hs, :]                                       # [R, nh', d_h + d_r]
     scores = np.einsum("rhd,thd->rht", qs, k) * scale          # [R, nh', S]
+    mask = np.zeros((len(rs), S))
+    if topk is not None:
+        tk = np.asarray(topk)
+        mask = np.stack([index_mask(S, tk[r]) for r in rs])   # the index mask of each query row
     if causal:
         t = np.arange(S)[None, :]
-        mask = np.where(t <= rs[:, None], 0.0, -np.inf)        # [R, S]
-        scores = scores + mask[:, None, :]
+        mask = mask + np.where(t <= rs[:, None], 0.0, -np.inf)  # [R, S]
+    scores = scores + mask[:, None, :]
     alpha = softmax(scores, axis=-1)
     return np.einsum("rht,thd->rhd", alpha, v)
 
@@ -281,3 +289,55 @@ def cache_append(kv_a, positions, d_c: int, d_r: int, gain=None, eps: float = 1e
     positions[b] (the decode reads row t as position t)."""
     x = _f64(kv_a)
     return rms_norm(x[:, :d_c], gain, eps), rope_interleaved(x[:, d_c:d_c + d_r], positions, base)
+
+
+# ----------------------------------------------------------------------------------------
+# Rows ranked next: several new tokens per decode, FP8 block-scaled wkv_b
+# ----------------------------------------------------------------------------------------
+
+def multi_token_decode(q_nope, q_pe, c_kv, k_r, w_kv_b, scale: float, d_v: int, topk=None):
+    """Absorbed decode of several new tokens of ONE sequence (the decode excerpt's "bshd" queries
+    with s > 1, e.g. speculative tokens).
+
+    q_nope [T, n_h, d_h], q_pe [T, n_h, d_r]; c_kv [L, d_c], k_r [L, d_r] hold the L cached rows,
+    the T new tokens being the last T of them (positions L - T .. L - 1).  The decode excerpt adds
+    no mask over s; the reading taken is the prefill excerpt's causal rule: query s attends rows
+    t <= L - T + s.  So T = 1 is the one-token decode, and the T results equal the last T rows of a
+    prefill over the same L rows.  ``topk`` [T, k] optionally holds each query's selected positions
+    (set semantics, then the causal rule), as in the sparse prefill.
+    Steps: q~ = absorb_q; s = scale (q~ . c_t + q_pe . k^R_t) + masks; alpha = softmax over t;
+    ctx = sum_t alpha c_t; o = out_up(ctx).  Returns a dict with q_tilde, ctx, lse and o, each
+    with the leading T axis.
+    """
+    q_nope, q_pe, c_kv, k_r = map(_f64, (q_nope, q_pe, c_kv, k_r))
+    T, n_h, d_h = q_nope.shape
+    L = c_kv.shape[0]
+    qt = absorb_q(q_nope, w_kv_b, n_h, d_h, d_v)                               # [T, n_h, d_c]
+    s = scale * (np.einsum("shc,tc->sht", qt, c_kv) + np.einsum("shr,tr->sht", q_pe, k_r))
+    pos = L - T + np.arange(T)                                                 # each query's position
+    mask = np.where(np.arange(L)[None, :] <= pos[:, None], 0.0, -np.inf)       # [T, L]
+    if topk is not None:
+        tk = np.asarray(topk)
+        mask = mask + np.stack([index_mask(L, tk[i]) for i in range(T)])
+    s = s + mask[:, None, :]
+    alpha = softmax(s, axis=-1)
+    ctx = np.einsum("sht,tc->shc", alpha, c_kv)
+    return {"q_tilde": qt, "ctx": ctx, "lse": _logsumexp(s, axis=-1),
+            "o": out_up(ctx, w_kv_b, n_h, d_h, d_v)}
+
+
+def fp8_block_scale_shape(out_features: int, in_features: int, block: int = 128):
+    """Scale grid of an FP8 weight ("Key-value down-projection", linear excerpt): one float32 scale
+    per block x block tile, ceil(out/block) x ceil(in/block)."""
+    return (out_features + block - 1) // block, (in_features + block - 1) // block
+
+
+def weight_dequant(w_q, scale, block: int = 128) -> np.ndarray:
+    """Dequantise an FP8 weight with one scale per 128 x 128 tile (linear excerpt: the scales are
+    quantisation metadata; "Value up-projection": the decode dequantises wkv_b once and uses it
+    unquantised): w[i, j] = w_q[i, j] * scale[i // block, j // block].  ``w_q`` may be a torch
+    float8 tensor (its values are read exactly)."""
+    w = _f64(w_q)
+    s = _f64(scale)
+    assert s.shape == fp8_block_scale_shape(w.shape[0], w.shape[1], block), "scale grid shape"
+    return w * s[np.arange(w.shape[0]) // block][:, np.arange(w.shape[1]) // block]
