@@ -235,7 +235,7 @@ static_assert(kBarOff + sizeof(Bars) + 1024 <= 232448, "dynamic shared memory ab
 // ------------------------------------------------------------------------------------------
 // Causal attention of the naive path ("Naive path": k = [k_nope; k_R broadcast], scores
 // q . k / sqrt(192), softmax over positions t <= s, output sum_t alpha_t v_t), per (sequence,
-// head, 128-query tile):
+// head, mirrored pair of 128-query tiles):
 //   * Q (128 x 192) is TMA-loaded once and read from shared memory by the score MMAs;
 //   * K tiles (128 keys: k_nope from the expanded rows, k_R shared by the heads) and V tiles stream
 //     through two 2-stage TMA rings (a K stage is released by its score MMA, a V stage by its P.V);
@@ -245,7 +245,7 @@ static_assert(kBarOff + sizeof(Bars) + 1024 <= 232448, "dynamic shared memory ab
 //   * online softmax in base 2, the running maximum raised (and O rescaled) only when it grows by
 //     more than 8.
 // ------------------------------------------------------------------------------------------
-constexpr int AT_TILE = 128;                      // queries per CTA, keys per tile
+constexpr int AT_TILE = 128;                      // queries per query tile, keys per key tile
 constexpr int AT_SLAB = AT_TILE * 128;            // 128 rows x 64 bf16 (128-byte swizzle)
 constexpr int AT_QOFF = 0;                        // Q: 3 slabs (q_nope 0-63, 64-127, q_pe)
 constexpr int AT_STAGES = 2;                      // K and V rings of two stages each
