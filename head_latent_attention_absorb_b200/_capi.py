@@ -49,6 +49,7 @@ SIGNATURES = {
                                   c_f32, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "mla_cache_append": (c_i32, [MLADims, c_i32, c_i32, c_vp, c_i64, c_vp, c_f32, c_f32, c_vp, c_i32,
                                  c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp]),
+    "mla_check_topk": (c_i32, [c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_vp]),
     "mla_clear_device_error": (c_i32, [c_vp, c_vp]),
     "mla_get_device_error": (c_i32, [c_vp, c_i32p]),
 }

@@ -200,6 +200,22 @@ def mla_cache_append(dims, kv_a: torch.Tensor, positions: torch.Tensor, c_kv: to
                                  k_r.stride(1), _ptr(dev_err), _stream(stream)), "mla_cache_append")
 
 
+def mla_check_topk(topk_idx: torch.Tensor, n_max: int, lengths: Optional[torch.Tensor] = None,
+                   dev_err: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Validate a top-k index array on the device: every index of row b inside [0, lengths[b])
+    (n_max when lengths is None) and listed once.  Sets MLA_ERR_INDEX / MLA_ERR_LENGTH in `dev_err`
+    (allocated zeroed here when not given), which is returned; read it with mla_get_device_error."""
+    if topk_idx.dtype != torch.int32 or not topk_idx.is_contiguous() or topk_idx.dim() != 2:
+        raise TypeError("topk_idx must be a contiguous int32 [B, topk] tensor")
+    if lengths is not None and (lengths.dtype != torch.int32 or not lengths.is_contiguous()):
+        raise TypeError("lengths must be a contiguous int32 tensor")
+    if dev_err is None:
+        dev_err = torch.zeros(1, dtype=torch.int32, device=topk_idx.device)
+    check(lib().mla_check_topk(topk_idx.shape[0], _ptr(topk_idx), topk_idx.shape[1], _ptr(lengths), int(n_max),
+                               _ptr(dev_err), _stream(stream)), "mla_check_topk")
+    return dev_err
+
+
 def mla_clear_device_error(dev_err: torch.Tensor, stream=None) -> None:
     check(lib().mla_clear_device_error(_ptr(dev_err), _stream(stream)), "mla_clear_device_error")
 

@@ -75,3 +75,59 @@ template cudaError_t cache_append_launch<float>(const AppendArgs&, cudaStream_t)
 template cudaError_t cache_append_launch<__nv_bfloat16>(const AppendArgs&, cudaStream_t);
 
 }  // namespace mla
+
+// ------------------------------------------------------------------------------------------
+// Top-k index validation (opt-in, outside the decode): the decode's gather reads each listed row
+// once, so a repeated index would count twice where the pages' scatter mask counts it once
+// ("Absorb key weights", decode excerpt: 0 scattered into a -inf row is a set).  One CTA per
+// sequence marks its indices in a shared-memory bitmap of the cache length; an index outside
+// [0, length) or one already marked raises MLA_ERR_INDEX.  Every bitmap access is behind the range
+// check, so no index can reach outside the bitmap.
+// ------------------------------------------------------------------------------------------
+namespace mla {
+namespace {
+
+constexpr int kCheckThreads = 256;
+
+__global__ void __launch_bounds__(kCheckThreads) check_topk_kernel(const int32_t* __restrict__ idx, int topk,
+                                                                   const int32_t* __restrict__ lengths, int n_max,
+                                                                   int32_t* err) {
+  extern __shared__ uint32_t seen[];  // ceil(n_max / 32) words
+  const int b = blockIdx.x;
+  const int words = (n_max + 31) >> 5;
+  for (int w = threadIdx.x; w < words; w += kCheckThreads) seen[w] = 0u;
+  __syncthreads();
+  const int len = lengths != nullptr ? lengths[b] : n_max;
+  if (len < 1 || len > n_max) {
+    if (threadIdx.x == 0) raise_error(err, MLA_ERR_LENGTH);
+    return;
+  }
+  const int32_t* row = idx + (int64_t)b * topk;
+  for (int i = threadIdx.x; i < topk; i += kCheckThreads) {
+    const int t = row[i];
+    if (t < 0 || t >= len) {
+      raise_error(err, MLA_ERR_INDEX);
+      continue;
+    }
+    const uint32_t bit = 1u << (t & 31);
+    if (atomicOr(&seen[t >> 5], bit) & bit) raise_error(err, MLA_ERR_INDEX);  // listed twice
+  }
+}
+
+}  // namespace
+
+size_t check_topk_smem_bytes(int n_max) { return (size_t)((n_max + 31) / 32) * sizeof(uint32_t); }
+
+cudaError_t check_topk_launch(int B, const int32_t* idx, int topk, const int32_t* lengths, int n_max, int32_t* err,
+                              cudaStream_t st) {
+  const size_t smem = check_topk_smem_bytes(n_max);
+  if (smem > 48 * 1024) {
+    const cudaError_t e = cudaFuncSetAttribute(check_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  check_topk_kernel<<<B, kCheckThreads, smem, st>>>(idx, topk, lengths, n_max, err);
+  return cudaGetLastError();
+}
+
+}  // namespace mla

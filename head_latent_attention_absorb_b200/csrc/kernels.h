@@ -27,6 +27,11 @@ int decode_simt_splits(int B, int n_keys_cap);
 template <typename T>
 cudaError_t cache_append_launch(const AppendArgs& a, cudaStream_t st);
 
+// ---- top-k index validation (range and distinctness per sequence) --------------------------
+size_t check_topk_smem_bytes(int n_max);
+cudaError_t check_topk_launch(int B, const int32_t* idx, int topk, const int32_t* lengths, int n_max, int32_t* err,
+                              cudaStream_t st);
+
 // ---- tcgen05 kernels (bf16, DeepSeek-V3 dimensions) ------------------------------------------
 size_t decode_tc_workspace(int B);
 cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st);

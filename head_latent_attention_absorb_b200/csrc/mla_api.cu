@@ -303,6 +303,18 @@ mla_status mla_cache_append(mla_dims dims, mla_dtype dtype, int32_t B, const voi
   return cuda_status(e, "mla_cache_append launch");
 }
 
+mla_status mla_check_topk(int32_t B, const int32_t* topk_idx, int32_t topk, const int32_t* lengths, int32_t n_max,
+                          int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  if (B <= 0 || topk <= 0 || n_max <= 0) return fail(MLA_ERR_INVALID_ARG, "B, topk and n_max must be positive");
+  if (!topk_idx || !dev_err) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (mla::check_topk_smem_bytes(n_max) > 232448)
+    return fail(MLA_ERR_UNSUPPORTED, "n_max %d: the position bitmap exceeds shared memory", n_max);
+  return cuda_status(mla::check_topk_launch(B, topk_idx, topk, lengths, n_max, dev_err,
+                                            static_cast<cudaStream_t>(stream)),
+                     "mla_check_topk launch");
+}
+
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream) {
   g_msg[0] = 0;
   if (!dev_err) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");

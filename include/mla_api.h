@@ -220,6 +220,22 @@ mla_status mla_cache_append(mla_dims dims, mla_dtype dtype, int32_t B,
                             void* k_r, int64_t kr_bstride, int64_t kr_rstride,
                             int32_t* dev_err, void* stream);
 
+/*
+ * mla_check_topk - opt-in validation of a top-k index array before a sparse decode.  The pages'
+ * mask ("Absorb key weights", decode excerpt) scatters 0 into a -inf row, so the selected
+ * positions form a set; the gather kernels read each listed row once, so distinct indices are
+ * their precondition.  This call checks it on the device, per sequence b:
+ *   topk_idx  DEVICE int32 [B, topk] contiguous
+ *   lengths   DEVICE int32 [B], or NULL for n_max everywhere
+ *   an index outside [0, lengths[b]) or listed twice in its row sets MLA_ERR_INDEX; a length
+ *   outside [1, n_max] sets MLA_ERR_LENGTH.  Nothing else is written.
+ *   n_max up to 1,859,584 (a bitmap of the positions in shared memory); larger returns
+ *   MLA_ERR_UNSUPPORTED.
+ * Asynchronous on `stream`; read the flag with mla_get_device_error.
+ */
+mla_status mla_check_topk(int32_t B, const int32_t* topk_idx, int32_t topk, const int32_t* lengths, int32_t n_max,
+                          int32_t* dev_err, void* stream);
+
 /* Zero the device flag (asynchronous on `stream`). */
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream);
 

@@ -110,6 +110,11 @@ def test_host_validation_codes(L):
                               FAKE, 8 * 64, 64, FAKE, 8 * 15, 15, None, None) == 1   # odd rotary width
     assert L.mla_cache_append(tiny, bf, 1, FAKE, 80, None, 1e-6, 1e4, FAKE, 8,
                               FAKE, 8 * 64, 64, FAKE, 8 * 16, 16, None, None) == 2   # bf16 outside DeepSeek dims
+    # top-k validation
+    assert L.mla_check_topk(0, FAKE, 8, None, 64, FAKE, None) == 1
+    assert L.mla_check_topk(2, None, 8, None, 64, FAKE, None) == 1
+    assert L.mla_check_topk(2, FAKE, 8, None, 64, None, None) == 1
+    assert L.mla_check_topk(2, FAKE, 8, None, 2_000_000, FAKE, None) == 2   # bitmap beyond shared memory
     assert L.mla_clear_device_error(None, None) == 1
     out = ctypes.c_int32(0)
     assert L.mla_get_device_error(None, ctypes.byref(out)) == 1
