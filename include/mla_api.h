@@ -1,7 +1,7 @@
 /*
  * mla_api.h - C ABI of libmla_b200.so: multi-head latent attention (MLA) for NVIDIA B200 (sm_100a).
  *
- * The four operations are the steps of DeepSeek-V3 / V3.2 MLA as the pages state them:
+ * The operations are the steps of DeepSeek-V3 / V3.2 MLA as the pages state them:
  *   mla_absorb_q       q~_i = (W^UK_i)^T q^C_i                       ("Absorb key weights", first einsum)
  *   mla_decode_absorb  softmax over cached positions of
  *                      scale (q~ . c^KV_t + q^R . k^R_t), weighted sum of c^KV_t
@@ -13,6 +13,8 @@
  *   mla_cache_append   the new token's latent (RMSNorm) and rotary key (RoPE) into the caches
  *                                                                    ("Key-value down-projection", mla-kv
  *                                                                     excerpt; "Key-value latent RMSNorm")
+ * plus one opt-in check of the sparse decode's precondition:
+ *   mla_check_topk     top-k indices in range and distinct per sequence (the mask is a set)
  *
  * Conventions shared by every call
  * --------------------------------
