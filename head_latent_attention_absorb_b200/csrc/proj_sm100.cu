@@ -172,18 +172,23 @@ size_t smem_bytes(bool absorb, int n_tile) {
   const int chunks = absorb ? kDH / 64 : kDC / 64, mbs = absorb ? Shape<true>::kMB : 1;
   return (size_t)chunks * (mbs * 128 * 64 * 2 + n_tile * 128) + 1024;
 }
+static_assert((kDC / 64) * (128 * 64 * 2 + 96 * 128) + 1024 <= 232448, "out_up tile above 227 KB of shared memory");
+static_assert((kDH / 64) * (2 * 128 * 64 * 2 + 256 * 128) + 1024 <= 232448, "absorb_q tile above 227 KB");
 
-// Batch rows per CTA: the whole batch up to 256 (one CTA per head and row block), else 256.
-int n_tile_for(int B) {
+// Batch rows per CTA: the whole batch up to the most that fits (one CTA per head and row block),
+// else that many per CTA.  absorb_q holds 2 x 2 weight chunks, so 256 rows fit; out_up holds all 8
+// chunks of its K = 512, and 8 x (16 KB + 128 B per row) stays within 227 KB only up to 96 rows.
+int n_tile_for(bool absorb, int B) {
+  const int cap = absorb ? 256 : 96;
   const int n = ((B + 15) / 16) * 16;
-  return n > 256 ? 256 : n;
+  return n > cap ? cap : n;
 }
 
 template <bool kAbsorb>
 cudaError_t launch(int B, const void* act, int64_t ld_head, const void* w, void* out, int32_t* err, cudaStream_t st) {
   Params p;
   memset(&p, 0, sizeof(p));
-  const int n_tile = n_tile_for(B);
+  const int n_tile = n_tile_for(kAbsorb, B);
   const int kfeat = kAbsorb ? kDH : kDC;
   {
     const uint64_t dims[2] = {(uint64_t)kDC, (uint64_t)kNH * kRowsPerHead};

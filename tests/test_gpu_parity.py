@@ -128,6 +128,24 @@ def test_v3_out_up(v3):
     check_close(o, O.out_up(ctx_t, v3["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v), torch.bfloat16, "out_up")
 
 
+@pytest.mark.parametrize("B", [97, 200, 300])
+def test_projections_large_batches(v3, B):
+    # batches past one CTA's tile: out_up takes 96 rows per CTA, absorb_q 256; rows on both sides of
+    # each tile boundary and the last row are checked against the oracle
+    cfg = V3_DECODE
+    rng = np.random.default_rng(B)
+    q_nope = torch.from_numpy(rng.standard_normal((B, cfg.n_h, cfg.d_h), dtype=np.float32)).to(torch.bfloat16)
+    ctx = torch.from_numpy(rng.standard_normal((B, cfg.n_h, cfg.d_c), dtype=np.float32) * 0.05).to(torch.bfloat16)
+    qt = api.mla_absorb_q(cfg.dims, q_nope.cuda(), v3["w_d"])
+    o = api.mla_out_up(cfg.dims, ctx.cuda(), v3["w_d"])
+    torch.cuda.synchronize()
+    rows = sorted({0, 95, 96, 191, 192, 255, 256, B - 1} & set(range(B)))
+    check_close(qt[rows], O.absorb_q(q_nope[rows], v3["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v), torch.bfloat16,
+                f"absorb_q B={B}")
+    check_close(o[rows], O.out_up(ctx[rows], v3["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v), torch.bfloat16,
+                f"out_up B={B}")
+
+
 def test_v3_whole_step_vs_oracle(v3):
     cfg = V3_DECODE
     qt, ctx, lse, o = gpu_step(v3, cfg.dims)
