@@ -172,6 +172,16 @@ def test_decode_ragged_tails(dev):
     check_decode_call(x, cfg.dims, torch.bfloat16)
 
 
+def test_decode_many_sequences(dev):
+    # more sequences than clusters (contiguous tile ranges, several sequences per cluster, split
+    # sequences at range ends) and more than 256 (the work plan re-reads tile counts from memory)
+    B = 300
+    lengths = torch.from_numpy(np.random.default_rng(300).integers(1, 301, B).astype(np.int32))
+    cfg = V3_DECODE.with_(B=B, n_max=300)
+    x = upload(make_decode_inputs(cfg, lengths=lengths), dev)
+    check_decode_call(x, cfg.dims, torch.bfloat16)
+
+
 def test_decode_separate_and_packed_layouts_agree(dev):
     cfg = V3_DECODE.with_(B=3, n_max=700)
     x = upload(make_decode_inputs(cfg, lengths=torch.tensor([700, 333, 64], dtype=torch.int32)), dev)
