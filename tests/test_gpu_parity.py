@@ -146,6 +146,22 @@ def test_projections_large_batches(v3, B):
                 f"out_up B={B}")
 
 
+def test_query_as_views_of_one_tensor(v3):
+    # the query projection yields [B, n_h, d_h + d_r]; q_nope and q_pe are strided views of it
+    # (row stride 192): the step must give the same bits as with contiguous copies
+    cfg = V3_DECODE
+    q = torch.cat([v3["q_nope_d"], v3["q_pe_d"]], dim=-1)
+    assert q.shape[-1] == cfg.d_h + cfg.d_r
+    qt_v = api.mla_absorb_q(cfg.dims, q[..., :cfg.d_h], v3["w_d"])
+    ctx_v = api.mla_decode_absorb(cfg.dims, qt_v, q[..., cfg.d_h:], v3["c_kv_d"], v3["k_r_d"], v3["len_d"], cfg.scale)
+    qt_c = api.mla_absorb_q(cfg.dims, v3["q_nope_d"].contiguous(), v3["w_d"])
+    ctx_c = api.mla_decode_absorb(cfg.dims, qt_c, v3["q_pe_d"].contiguous(), v3["c_kv_d"], v3["k_r_d"], v3["len_d"],
+                                  cfg.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(qt_v, qt_c)
+    assert torch.equal(ctx_v, ctx_c)
+
+
 def test_v3_whole_step_vs_oracle(v3):
     cfg = V3_DECODE
     qt, ctx, lse, o = gpu_step(v3, cfg.dims)
