@@ -128,40 +128,6 @@ def test_v3_out_up(v3):
     check_close(o, O.out_up(ctx_t, v3["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v), torch.bfloat16, "out_up")
 
 
-@pytest.mark.parametrize("B", [97, 200, 300])
-def test_projections_large_batches(v3, B):
-    # batches past one CTA's tile: out_up takes 96 rows per CTA, absorb_q 256; rows on both sides of
-    # each tile boundary and the last row are checked against the oracle
-    cfg = V3_DECODE
-    rng = np.random.default_rng(B)
-    q_nope = torch.from_numpy(rng.standard_normal((B, cfg.n_h, cfg.d_h), dtype=np.float32)).to(torch.bfloat16)
-    ctx = torch.from_numpy(rng.standard_normal((B, cfg.n_h, cfg.d_c), dtype=np.float32) * 0.05).to(torch.bfloat16)
-    qt = api.mla_absorb_q(cfg.dims, q_nope.cuda(), v3["w_d"])
-    o = api.mla_out_up(cfg.dims, ctx.cuda(), v3["w_d"])
-    torch.cuda.synchronize()
-    rows = sorted({0, 95, 96, 191, 192, 255, 256, B - 1} & set(range(B)))
-    check_close(qt[rows], O.absorb_q(q_nope[rows], v3["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v), torch.bfloat16,
-                f"absorb_q B={B}")
-    check_close(o[rows], O.out_up(ctx[rows], v3["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v), torch.bfloat16,
-                f"out_up B={B}")
-
-
-def test_query_as_views_of_one_tensor(v3):
-    # the query projection yields [B, n_h, d_h + d_r]; q_nope and q_pe are strided views of it
-    # (row stride 192): the step must give the same bits as with contiguous copies
-    cfg = V3_DECODE
-    q = torch.cat([v3["q_nope_d"], v3["q_pe_d"]], dim=-1)
-    assert q.shape[-1] == cfg.d_h + cfg.d_r
-    qt_v = api.mla_absorb_q(cfg.dims, q[..., :cfg.d_h], v3["w_d"])
-    ctx_v = api.mla_decode_absorb(cfg.dims, qt_v, q[..., cfg.d_h:], v3["c_kv_d"], v3["k_r_d"], v3["len_d"], cfg.scale)
-    qt_c = api.mla_absorb_q(cfg.dims, v3["q_nope_d"].contiguous(), v3["w_d"])
-    ctx_c = api.mla_decode_absorb(cfg.dims, qt_c, v3["q_pe_d"].contiguous(), v3["c_kv_d"], v3["k_r_d"], v3["len_d"],
-                                  cfg.scale)
-    torch.cuda.synchronize()
-    assert torch.equal(qt_v, qt_c)
-    assert torch.equal(ctx_v, ctx_c)
-
-
 def test_v3_whole_step_vs_oracle(v3):
     cfg = V3_DECODE
     qt, ctx, lse, o = gpu_step(v3, cfg.dims)
@@ -185,16 +151,6 @@ TAIL_LENGTHS = [1, 2, 63, 64, 65, 127, 128, 129, 255, 1000, 1024, 1100]
 def test_decode_ragged_tails(dev):
     cfg = V3_DECODE.with_(B=len(TAIL_LENGTHS), n_max=1100)
     x = upload(make_decode_inputs(cfg, lengths=torch.tensor(TAIL_LENGTHS, dtype=torch.int32)), dev)
-    check_decode_call(x, cfg.dims, torch.bfloat16)
-
-
-def test_decode_many_sequences(dev):
-    # more sequences than clusters (contiguous tile ranges, several sequences per cluster, split
-    # sequences at range ends) and more than 256 (the work plan re-reads tile counts from memory)
-    B = 300
-    lengths = torch.from_numpy(np.random.default_rng(300).integers(1, 301, B).astype(np.int32))
-    cfg = V3_DECODE.with_(B=B, n_max=300)
-    x = upload(make_decode_inputs(cfg, lengths=lengths), dev)
     check_decode_call(x, cfg.dims, torch.bfloat16)
 
 
