@@ -44,12 +44,17 @@ SIGNATURES = {
                                          c_vp, c_i64, c_i64, c_vp, c_i64, c_i64,
                                          c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_vp]),
     "mla_out_up": (c_i32, [MLADims, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
+    "mla_absorb_q_fp8": (c_i32, [MLADims, c_i32, c_vp, c_i64, c_vp, c_vp, c_vp, c_vp, c_vp]),
+    "mla_out_up_fp8": (c_i32, [MLADims, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp]),
     "mla_prefill_workspace_size": (c_sz, [MLADims, c_i32, c_i32, c_i32]),
     "mla_prefill_naive": (c_i32, [MLADims, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp,
                                   c_f32, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "mla_cache_append": (c_i32, [MLADims, c_i32, c_i32, c_vp, c_i64, c_vp, c_f32, c_f32, c_vp, c_i32,
                                  c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_vp]),
     "mla_check_topk": (c_i32, [c_i32, c_vp, c_i32, c_vp, c_i32, c_vp, c_vp]),
+    "mla_prefill_sparse_workspace_size": (c_sz, [MLADims, c_i32, c_i32, c_i32]),
+    "mla_prefill_sparse": (c_i32, [MLADims, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp,
+                                   c_f32, c_vp, c_i32, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "mla_clear_device_error": (c_i32, [c_vp, c_vp]),
     "mla_get_device_error": (c_i32, [c_vp, c_i32p]),
 }

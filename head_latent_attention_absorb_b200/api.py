@@ -147,6 +147,40 @@ def mla_out_up(dims, ctx: torch.Tensor, w_kv_b: torch.Tensor, out: Optional[torc
     return out
 
 
+def mla_absorb_q_fp8(dims, q_nope: torch.Tensor, w_fp8: torch.Tensor, w_scale: torch.Tensor,
+                     q_tilde: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """mla_absorb_q with an e4m3 wkv_b (w_fp8, torch.float8_e4m3fn) and its fp32 128 x 128 block
+    scales (w_scale [rows / 128, d_c / 128])."""
+    d = _dims(dims)
+    B = q_nope.shape[0]
+    ldq = _headrows(q_nope, "q_nope")
+    if w_fp8.dtype != torch.float8_e4m3fn or w_scale.dtype != torch.float32 or not w_scale.is_contiguous():
+        raise TypeError("w_fp8 must be float8_e4m3fn and w_scale contiguous float32")
+    if q_tilde is None:
+        q_tilde = torch.empty((B, d.n_h, d.d_c), dtype=torch.bfloat16, device=q_nope.device)
+    check(lib().mla_absorb_q_fp8(d, B, _ptr(q_nope), ldq, _ptr(w_fp8), _ptr(w_scale), _ptr(q_tilde), _ptr(dev_err),
+                                 _stream(stream)), "mla_absorb_q_fp8")
+    return q_tilde
+
+
+def mla_out_up_fp8(dims, ctx: torch.Tensor, w_fp8: torch.Tensor, w_scale: torch.Tensor,
+                   out: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """mla_out_up with an e4m3 wkv_b and its fp32 128 x 128 block scales."""
+    d = _dims(dims)
+    B = ctx.shape[0]
+    if not ctx.is_contiguous():
+        raise ValueError("ctx must be contiguous")
+    if w_fp8.dtype != torch.float8_e4m3fn or w_scale.dtype != torch.float32 or not w_scale.is_contiguous():
+        raise TypeError("w_fp8 must be float8_e4m3fn and w_scale contiguous float32")
+    if out is None:
+        out = torch.empty((B, d.n_h, d.d_v), dtype=torch.bfloat16, device=ctx.device)
+    check(lib().mla_out_up_fp8(d, B, _ptr(ctx), _ptr(w_fp8), _ptr(w_scale), _ptr(out), _ptr(dev_err),
+                               _stream(stream)), "mla_out_up_fp8")
+    return out
+
+
 def mla_prefill_workspace_size(dims, dtype: torch.dtype, B: int, S: int) -> int:
     return int(lib().mla_prefill_workspace_size(_dims(dims), _DT[dtype], B, S))
 
@@ -214,6 +248,34 @@ def mla_check_topk(topk_idx: torch.Tensor, n_max: int, lengths: Optional[torch.T
     check(lib().mla_check_topk(topk_idx.shape[0], _ptr(topk_idx), topk_idx.shape[1], _ptr(lengths), int(n_max),
                                _ptr(dev_err), _stream(stream)), "mla_check_topk")
     return dev_err
+
+
+def mla_prefill_sparse(dims, q: torch.Tensor, c_kv: torch.Tensor, k_r: torch.Tensor, w_kv_b: torch.Tensor,
+                       scale: float, topk_idx: torch.Tensor, out: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """Sparse prefill: as mla_prefill_naive (causal), each query row attending only the positions
+    its row of topk_idx (int32 [B, S, k]) selects."""
+    d = _dims(dims)
+    B, S = c_kv.shape[0], c_kv.shape[1]
+    if not q.is_contiguous():
+        raise ValueError("q must be contiguous")
+    for t, n in ((c_kv, "c_kv"), (k_r, "k_r")):
+        _rows(t, n)
+        if t.stride(0) != S * t.stride(1):
+            raise ValueError(f"{n}: rows of consecutive sequences must be evenly strided")
+    if topk_idx.dtype != torch.int32 or not topk_idx.is_contiguous() or tuple(topk_idx.shape[:2]) != (B, S):
+        raise TypeError("topk_idx must be a contiguous int32 [B, S, k] tensor")
+    if out is None:
+        out = torch.empty((B, S, d.n_h, d.d_v), dtype=q.dtype, device=q.device)
+    if workspace is None:
+        nbytes = int(lib().mla_prefill_sparse_workspace_size(d, _dt(q), B, S))
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=q.device)
+    check(lib().mla_prefill_sparse(d, _dt(q), B, S, _ptr(q), _ptr(c_kv), c_kv.stride(1), _ptr(k_r), k_r.stride(1),
+                                   _ptr(w_kv_b), float(scale), _ptr(topk_idx), topk_idx.shape[2], _ptr(out),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(dev_err),
+                                   _stream(stream)), "mla_prefill_sparse")
+    return out
 
 
 def mla_clear_device_error(dev_err: torch.Tensor, stream=None) -> None:

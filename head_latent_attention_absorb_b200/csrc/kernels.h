@@ -37,8 +37,16 @@ size_t decode_tc_workspace(int B);
 cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st);
 cudaError_t absorb_q_tc_launch(int B, const void* q_nope, int64_t ldq, const void* w, void* q_tilde, cudaStream_t st);
 cudaError_t out_up_tc_launch(int B, const void* ctx, const void* w, void* out, cudaStream_t st);
+cudaError_t absorb_q_fp8_tc_launch(int B, const void* q_nope, int64_t ldq, const void* w_fp8, const float* scale,
+                                   void* q_tilde, int32_t* err, cudaStream_t st);
+cudaError_t out_up_fp8_tc_launch(int B, const void* ctx, const void* w_fp8, const float* scale, void* out,
+                                 int32_t* err, cudaStream_t st);
 cudaError_t expand_tc_launch(const PrefillArgs& a, cudaStream_t st);
 cudaError_t attn_tc_launch(const PrefillArgs& a, cudaStream_t st);
+size_t sparse_prefill_scratch_bytes(int B, int S);
+cudaError_t sparse_masks_launch(const PrefillArgs& a, const int32_t* topk, int k, void* scratch, int32_t* err,
+                                cudaStream_t st);
+cudaError_t attn_sparse_tc_launch(const PrefillArgs& a, const void* scratch, int32_t* err, cudaStream_t st);
 template <typename T>
 cudaError_t prefill_attn_simt_launch(const PrefillArgs& a, cudaStream_t st);
 size_t decode_static_scratch_bytes();

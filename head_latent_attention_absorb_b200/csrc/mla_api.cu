@@ -224,6 +224,35 @@ mla_status mla_out_up(mla_dims dims, mla_dtype dtype, int32_t B, const void* ctx
   return cuda_status(e, "mla_out_up launch");
 }
 
+mla_status mla_absorb_q_fp8(mla_dims dims, int32_t B, const void* q_nope, int64_t ldq, const void* w_fp8,
+                            const float* w_scale, void* q_tilde, int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, MLA_BF16));
+  if (B <= 0) return fail(MLA_ERR_INVALID_ARG, "B must be positive");
+  if (!q_nope || !w_fp8 || !w_scale || !q_tilde) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (ldq < dims.d_h) return fail(MLA_ERR_INVALID_ARG, "ldq smaller than d_h");
+  MLA_TRY(check_bf16_ptr(MLA_BF16, q_nope, "q_nope"));
+  MLA_TRY(check_bf16_ptr(MLA_BF16, w_fp8, "w_fp8"));
+  MLA_TRY(check_bf16_ptr(MLA_BF16, q_tilde, "q_tilde"));
+  MLA_TRY(check_bf16_stride(MLA_BF16, ldq, "ldq"));
+  return cuda_status(mla::absorb_q_fp8_tc_launch(B, q_nope, ldq, w_fp8, w_scale, q_tilde, dev_err,
+                                                 static_cast<cudaStream_t>(stream)),
+                     "mla_absorb_q_fp8 launch");
+}
+
+mla_status mla_out_up_fp8(mla_dims dims, int32_t B, const void* ctx, const void* w_fp8, const float* w_scale,
+                          void* out, int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, MLA_BF16));
+  if (B <= 0) return fail(MLA_ERR_INVALID_ARG, "B must be positive");
+  if (!ctx || !w_fp8 || !w_scale || !out) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  MLA_TRY(check_bf16_ptr(MLA_BF16, ctx, "ctx"));
+  MLA_TRY(check_bf16_ptr(MLA_BF16, w_fp8, "w_fp8"));
+  MLA_TRY(check_bf16_ptr(MLA_BF16, out, "out"));
+  return cuda_status(mla::out_up_fp8_tc_launch(B, ctx, w_fp8, w_scale, out, dev_err, static_cast<cudaStream_t>(stream)),
+                     "mla_out_up_fp8 launch");
+}
+
 size_t mla_prefill_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S) {
   if (check_dims(dims, dtype) != MLA_OK || B <= 0 || S <= 0) return 0;
   const size_t es = dtype == MLA_BF16 ? 2 : 4;
@@ -313,6 +342,49 @@ mla_status mla_check_topk(int32_t B, const int32_t* topk_idx, int32_t topk, cons
   return cuda_status(mla::check_topk_launch(B, topk_idx, topk, lengths, n_max, dev_err,
                                             static_cast<cudaStream_t>(stream)),
                      "mla_check_topk launch");
+}
+
+size_t mla_prefill_sparse_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S) {
+  const size_t dense = mla_prefill_workspace_size(dims, dtype, B, S);
+  if (dense == 0 || dtype != MLA_BF16) return 0;
+  return ((dense + 255) & ~(size_t)255) + mla::sparse_prefill_scratch_bytes(B, S);
+}
+
+mla_status mla_prefill_sparse(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S, const void* q, const void* c_kv,
+                              int64_t ckv_rstride, const void* k_r, int64_t kr_rstride, const void* w_kv_b,
+                              float scale, const int32_t* topk_idx, int32_t topk, void* out, void* workspace,
+                              size_t ws_bytes, int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  MLA_TRY(check_dims(dims, dtype));
+  if (dtype != MLA_BF16) return fail(MLA_ERR_UNSUPPORTED, "mla_prefill_sparse covers bf16 only");
+  if (B <= 0 || S <= 0 || topk <= 0) return fail(MLA_ERR_INVALID_ARG, "B, S and topk must be positive");
+  if (!q || !c_kv || !k_r || !w_kv_b || !out || !topk_idx) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (ckv_rstride < dims.d_c || kr_rstride < dims.d_r) return fail(MLA_ERR_INVALID_ARG, "row stride too small");
+  if (!(scale > 0.f)) return fail(MLA_ERR_INVALID_ARG, "scale must be positive");
+  MLA_TRY(check_bf16_ptr(dtype, q, "q"));
+  MLA_TRY(check_bf16_ptr(dtype, c_kv, "c_kv"));
+  MLA_TRY(check_bf16_ptr(dtype, k_r, "k_r"));
+  MLA_TRY(check_bf16_ptr(dtype, w_kv_b, "w_kv_b"));
+  MLA_TRY(check_bf16_ptr(dtype, out, "out"));
+  MLA_TRY(check_bf16_stride(dtype, ckv_rstride, "ckv_rstride"));
+  MLA_TRY(check_bf16_stride(dtype, kr_rstride, "kr_rstride"));
+  const size_t need = mla_prefill_sparse_workspace_size(dims, dtype, B, S);
+  if (!workspace || ws_bytes < need)
+    return fail(MLA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace ? ws_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(MLA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+  if ((size_t)16 * ((S + 127) / 128) > 48 * 1024) return fail(MLA_ERR_UNSUPPORTED, "S too long for the row bitmap");
+  mla::PrefillArgs a;
+  a.n_h = dims.n_h; a.d_c = dims.d_c; a.d_r = dims.d_r; a.d_h = dims.d_h; a.d_v = dims.d_v;
+  a.B = B; a.S = S; a.causal = 1;
+  a.q = q; a.c_kv = c_kv; a.ckv_r = ckv_rstride; a.k_r = k_r; a.kr_r = kr_rstride; a.w = w_kv_b;
+  a.scale = scale; a.out = out; a.kv = workspace;
+  void* scratch = static_cast<uint8_t*>(workspace) + ((mla_prefill_workspace_size(dims, dtype, B, S) + 255) & ~(size_t)255);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = mla::sparse_masks_launch(a, topk_idx, topk, scratch, dev_err, st);
+  if (e == cudaSuccess) e = mla::expand_tc_launch(a, st);
+  if (e == cudaSuccess) e = mla::attn_sparse_tc_launch(a, scratch, dev_err, st);
+  return cuda_status(e, "mla_prefill_sparse launch");
 }
 
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream) {

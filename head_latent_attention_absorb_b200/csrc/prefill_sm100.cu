@@ -266,6 +266,12 @@ struct AttnParams {
   int B, S, H, n_qt, causal;
   float scale_log2;
   int32_t* err;
+  // sparse variant: each query row's selected key positions (already cut to t <= s) as a bitmap,
+  // and per (sequence, query tile) the compact list of key tiles any of its rows selects
+  const uint32_t* bitmap;   // [B][S][row_words]
+  int row_words;            // 4 * n_qt (128 bits per key tile)
+  const int32_t* tile_list; // [B][n_qt][n_qt]
+  const int32_t* tile_count;// [B][n_qt]
 };
 
 struct AttnBars {
@@ -289,6 +295,7 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+template <bool kSparse>
 __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_constant__ AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -305,7 +312,14 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
   const int pi = idx % n_pairs, h = (idx / n_pairs) % p.H, b = idx / (n_pairs * p.H);
   const int n_items = (p.n_qt - 1 - pi != pi) ? 2 : 1;
   auto item_qt = [&](int it) { return it == 0 ? p.n_qt - 1 - pi : pi; };
-  auto item_nkv = [&](int it) { return p.causal ? item_qt(it) + 1 : p.n_qt; };  // key tiles attended
+  // key tiles attended by query tile `it`, and the j-th of them
+  auto item_nkv = [&](int it) {
+    if (kSparse) return p.tile_count[b * p.n_qt + item_qt(it)];
+    return p.causal ? item_qt(it) + 1 : p.n_qt;
+  };
+  auto key_tile = [&](int it, int j) {
+    return kSparse ? p.tile_list[((int64_t)b * p.n_qt + item_qt(it)) * p.n_qt + j] : j;
+  };
 
   griddep_launch_dependents();
   if (threadIdx.x == 0) {
@@ -354,7 +368,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       const uint32_t qb = smem_u32(&bs.q_tma);
       const int n_kv0 = item_nkv(0);
       const int G = n_kv0 + (n_items > 1 ? item_nkv(1) : 0);
-      auto key_row = [&](int g) { return AT_TILE * (g < n_kv0 ? g : g - n_kv0); };
+      auto key_row = [&](int g) { return AT_TILE * (g < n_kv0 ? key_tile(0, g) : key_tile(1, g - n_kv0)); };
       bool ok = true;
       int nk = 0, nv = 0;  // K and V tiles issued
       mbar_arrive_expect_tx(qb, 3 * AT_SLAB);
@@ -495,7 +509,7 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
         if (!wait_all(smem_u32(&bs.s_full[g % AT_SBUF]), (g / AT_SBUF) & 1u)) break;
         tc_fence_after();
         const uint32_t tS = tmem + lane_off + AT_COL_S + 128 * (g % AT_SBUF);
-        const int key0 = AT_TILE * j;
+        const int key0 = AT_TILE * key_tile(it, j);
         // keys of this tile this row may attend: below the sequence length and (causal) <= q_pos
         const int lim = p.causal ? min(p.S - 1, q_pos) : p.S - 1;
         const int nvalid = lim - key0 + 1;  // keys 0 .. nvalid-1 of the tile are valid
@@ -506,7 +520,19 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
         tmem_ld_wait();
         // masked keys (past the row's causal limit or the sequence end; only the diagonal and the
         // last tile have any) become -inf: they leave the maximum alone and 2^-inf = 0
-        if (nvalid < AT_TILE) {
+        if (kSparse) {
+          // the row's selected keys of this tile: 128 bits (causal and length already applied);
+          // rows past the sequence end select nothing
+          uint4 bits = make_uint4(0u, 0u, 0u, 0u);
+          if (q_pos < p.S)
+            bits = *reinterpret_cast<const uint4*>(p.bitmap + ((int64_t)b * p.S + q_pos) * p.row_words + (key0 >> 5));
+          const uint32_t bw[4] = {bits.x, bits.y, bits.z, bits.w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              sv[c][k] = (bw[c] >> k) & 1u ? sv[c][k] : 0xff800000u;
+        } else if (nvalid < AT_TILE) {
 #pragma unroll
           for (int c = 0; c < 4; ++c)
 #pragma unroll
@@ -546,14 +572,17 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
         }
         // P = 2^(s scale_log2 - m) in bf16, written over the scores it came from (chunk c of P takes
         // columns [16c, 16c + 16); the whole row is already in registers)
+        // a sparse row with no selected key so far keeps m = -inf: its scores are all -inf, so any
+        // finite reference gives P = 0 (a -inf reference would give 2^NaN)
+        const float m_ref = (kSparse && m_run == -INFINITY) ? 0.f : m_run;
         float lsv[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int k = 0; k < 16; ++k) {
-            const float p0 = ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k]), p.scale_log2, -m_run));
-            const float p1 = ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k + 1]), p.scale_log2, -m_run));
+            const float p0 = ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k]), p.scale_log2, -m_ref));
+            const float p1 = ex2f_approx(fmaf(__uint_as_float(sv[c][2 * k + 1]), p.scale_log2, -m_ref));
             lsv[k & 3] += p0 + p1;
             pk[k] = pack_bf16x2(p0, p1);
           }
@@ -570,7 +599,10 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
       // has completed
       if (n_kv >= 1 && wait_all(smem_u32(&bs.pv_done[(g - 1) % AT_SBUF]), ((g - 1) / AT_SBUF) & 1u)) {
         tc_fence_after();
-        const float inv = 1.f / l_run;
+        // a sparse row that selected no visible key has no softmax: it is written as zeros and flagged
+        const bool empty_row = kSparse && !(l_run > 0.f);
+        if (empty_row && q_pos < p.S) raise_error(p.err, MLA_ERR_INDEX);
+        const float inv = empty_row ? 0.f : 1.f / l_run;
 #pragma unroll 1
         for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
@@ -599,6 +631,55 @@ __global__ void __launch_bounds__(AT_THREADS, 1) attn_kernel(const __grid_consta
 }
 
 size_t attn_smem_bytes() { return (size_t)AT_BAROFF + sizeof(AttnBars) + 1024; }
+
+// ---- sparse prefill: each query row's top-k set -> bitmap rows and per-query-tile key-tile lists ----
+// One CTA per (row s, sequence b): the row's selected positions t <= s as bits (a set: repeats
+// merge), written out as 4 words per key tile, and the key tiles holding any selected position
+// marked for the row's query tile.  `activity` must be zero on entry.
+__global__ void __launch_bounds__(128) sparse_rows_kernel(const int32_t* __restrict__ topk, int k, int S, int n_qt,
+                                                         uint32_t* __restrict__ bitmap, int32_t* __restrict__ activity,
+                                                         int32_t* err) {
+  extern __shared__ uint32_t bits[];  // 4 * n_qt words
+  const int s = blockIdx.x, b = blockIdx.y;
+  const int words = 4 * n_qt;
+  for (int w = threadIdx.x; w < words; w += blockDim.x) bits[w] = 0u;
+  __syncthreads();
+  const int32_t* row = topk + ((int64_t)b * S + s) * k;
+  for (int i = threadIdx.x; i < k; i += blockDim.x) {
+    const int t = row[i];
+    if (t < 0 || t >= S) {
+      raise_error(err, MLA_ERR_INDEX);
+      continue;
+    }
+    if (t > s) continue;  // the causal mask removes it
+    atomicOr(&bits[t >> 5], 1u << (t & 31));
+  }
+  __syncthreads();
+  uint32_t* dst = bitmap + ((int64_t)b * S + s) * words;
+  for (int w = threadIdx.x; w < words; w += blockDim.x) dst[w] = bits[w];
+  const int qt = s / AT_TILE;
+  for (int kt = threadIdx.x; kt < n_qt; kt += blockDim.x)
+    if (bits[4 * kt] | bits[4 * kt + 1] | bits[4 * kt + 2] | bits[4 * kt + 3])
+      activity[((int64_t)b * n_qt + qt) * n_qt + kt] = 1;  // every writer stores the same 1
+}
+
+// One warp per (query tile, sequence): the active key tiles in increasing order, and their count.
+__global__ void __launch_bounds__(32) sparse_lists_kernel(const int32_t* __restrict__ activity, int n_qt,
+                                                         int32_t* __restrict__ tile_list,
+                                                         int32_t* __restrict__ tile_count) {
+  const int qt = blockIdx.x, b = blockIdx.y, lane = threadIdx.x;
+  const int32_t* act = activity + ((int64_t)b * n_qt + qt) * n_qt;
+  int32_t* list = tile_list + ((int64_t)b * n_qt + qt) * n_qt;
+  int count = 0;
+  for (int base = 0; base < n_qt; base += 32) {
+    const int kt = base + lane;
+    const bool on = kt < n_qt && act[kt] != 0;
+    const unsigned m = __ballot_sync(0xffffffffu, on);
+    if (on) list[count + __popc(m & ((1u << lane) - 1u))] = kt;
+    count += __popc(m);
+  }
+  if (lane == 0) tile_count[b * n_qt + qt] = count;
+}
 static_assert(AT_BAROFF + sizeof(AttnBars) + 1024 <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
 }  // namespace prefill_tc
 
@@ -641,30 +722,25 @@ cudaError_t expand_tc_launch(const PrefillArgs& a, cudaStream_t st) {
   return launch_pdl(expand_kernel, dim3(grid), dim3(kThreads), smem, st, p);
 }
 
-// Causal (or full) attention of the naive path over the expanded rows in a.kv, bf16, DeepSeek dims.
-cudaError_t attn_tc_launch(const PrefillArgs& a, cudaStream_t st) {
-  using namespace prefill_tc;
-  AttnParams p;
+namespace prefill_tc {
+static bool attn_params(const PrefillArgs& a, AttnParams& p) {
   memset(&p, 0, sizeof(p));
   const uint64_t H = (uint64_t)a.n_h, S = (uint64_t)a.S, B = (uint64_t)a.B;
   const uint64_t dq = (uint64_t)(a.d_h + a.d_r), dkv = (uint64_t)(a.d_h + a.d_v);
   {
     const uint64_t dims[4] = {dq, H, S, B}, strides[3] = {dq * 2, H * dq * 2, S * H * dq * 2};
     const uint32_t box[4] = {64, 1, AT_TILE, 1};
-    if (!make_tensor_map_bf16(&p.tm_q, a.q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&p.tm_q, a.q, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return false;
   }
   {
     const uint64_t dims[4] = {dkv, H, S, B}, strides[3] = {dkv * 2, H * dkv * 2, S * H * dkv * 2};
     const uint32_t box[4] = {64, 1, AT_TILE, 1};
-    if (!make_tensor_map_bf16(&p.tm_kv, a.kv, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&p.tm_kv, a.kv, 4, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return false;
   }
   {
     const uint64_t dims[3] = {(uint64_t)a.d_r, S, B}, strides[2] = {(uint64_t)a.kr_r * 2, S * (uint64_t)a.kr_r * 2};
     const uint32_t box[3] = {64, AT_TILE, 1};
-    if (!make_tensor_map_bf16(&p.tm_kr, a.k_r, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
-      return cudaErrorInvalidValue;
+    if (!make_tensor_map_bf16(&p.tm_kr, a.k_r, 3, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B)) return false;
   }
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.B = a.B;
@@ -674,10 +750,70 @@ cudaError_t attn_tc_launch(const PrefillArgs& a, cudaStream_t st) {
   p.causal = a.causal;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.err = nullptr;
+  return true;
+}
+
+template <bool kSparse>
+static cudaError_t attn_launch(const AttnParams& p, int B, int H, cudaStream_t st) {
   const size_t smem = attn_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  cudaError_t e = cudaFuncSetAttribute(attn_kernel<kSparse>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_kernel, dim3((unsigned)((p.n_qt + 1) / 2 * a.B * a.n_h)), dim3(AT_THREADS), smem, st, p);
+  return launch_pdl(attn_kernel<kSparse>, dim3((unsigned)((p.n_qt + 1) / 2 * B * H)), dim3(AT_THREADS), smem, st,
+                    p);
+}
+}  // namespace prefill_tc
+
+// Causal (or full) attention of the naive path over the expanded rows in a.kv, bf16, DeepSeek dims.
+cudaError_t attn_tc_launch(const PrefillArgs& a, cudaStream_t st) {
+  using namespace prefill_tc;
+  AttnParams p;
+  if (!attn_params(a, p)) return cudaErrorInvalidValue;
+  return attn_launch<false>(p, a.B, a.n_h, st);
+}
+
+size_t sparse_prefill_scratch_bytes(int B, int S) {
+  const int n_qt = (S + prefill_tc::AT_TILE - 1) / prefill_tc::AT_TILE;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  return up((size_t)B * S * 4 * n_qt * 4) + 2 * up((size_t)B * n_qt * n_qt * 4) + up((size_t)B * n_qt * 4);
+}
+
+// The masks of the sparse prefill (bitmap rows, key-tile lists) into `scratch`; launched before the
+// expansion, so they are complete before the attention starts.
+cudaError_t sparse_masks_launch(const PrefillArgs& a, const int32_t* topk, int k, void* scratch, int32_t* err,
+                                cudaStream_t st) {
+  using namespace prefill_tc;
+  const int n_qt = (a.S + AT_TILE - 1) / AT_TILE;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  uint32_t* bitmap = reinterpret_cast<uint32_t*>(base);
+  int32_t* activity = reinterpret_cast<int32_t*>(base + up((size_t)a.B * a.S * 4 * n_qt * 4));
+  int32_t* list = activity + up((size_t)a.B * n_qt * n_qt * 4) / 4;
+  int32_t* count = list + up((size_t)a.B * n_qt * n_qt * 4) / 4;
+  cudaError_t e = cudaMemsetAsync(activity, 0, (size_t)a.B * n_qt * n_qt * 4, st);
+  if (e != cudaSuccess) return e;
+  sparse_rows_kernel<<<dim3(a.S, a.B), 128, (size_t)16 * n_qt, st>>>(topk, k, a.S, n_qt, bitmap, activity, err);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  sparse_lists_kernel<<<dim3(n_qt, a.B), 32, 0, st>>>(activity, n_qt, list, count);
+  return cudaGetLastError();
+}
+
+// Attention of the sparse prefill: each query row attends its selected positions t <= s.
+cudaError_t attn_sparse_tc_launch(const PrefillArgs& a, const void* scratch, int32_t* err, cudaStream_t st) {
+  using namespace prefill_tc;
+  AttnParams p;
+  if (!attn_params(a, p)) return cudaErrorInvalidValue;
+  const int n_qt = p.n_qt;
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  const uint8_t* base = static_cast<const uint8_t*>(scratch);
+  p.bitmap = reinterpret_cast<const uint32_t*>(base);
+  p.row_words = 4 * n_qt;
+  const int32_t* activity = reinterpret_cast<const int32_t*>(base + up((size_t)a.B * a.S * 4 * n_qt * 4));
+  p.tile_list = activity + up((size_t)a.B * n_qt * n_qt * 4) / 4;
+  p.tile_count = p.tile_list + up((size_t)a.B * n_qt * n_qt * 4) / 4;
+  p.causal = 1;
+  p.err = err;
+  return attn_launch<true>(p, a.B, a.n_h, st);
 }
 
 }  // namespace mla

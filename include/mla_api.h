@@ -173,6 +173,22 @@ mla_status mla_out_up(mla_dims dims, mla_dtype dtype, int32_t B,
                       const void* ctx, const void* w_kv_b, void* out, void* stream);
 
 /*
+ * mla_absorb_q_fp8 / mla_out_up_fp8 - mla_absorb_q and mla_out_up with an FP8 wkv_b ("Key-value
+ * down-projection", linear excerpt: an FP8 weight carries one float32 scale per 128 x 128 block;
+ * the decode uses the dequantised matrix, "Value up-projection").
+ *   w_fp8    e4m3 [n_h*(d_h+d_v), d_c] row-major, 16-byte aligned
+ *   w_scale  DEVICE fp32 [ceil(n_h*(d_h+d_v)/128), ceil(d_c/128)] row-major: the weight is
+ *            w[i, j] = w_fp8[i, j] * w_scale[i / 128, j / 128]
+ *   The weight is read as FP8 and dequantised on chip to bf16 (each value times its block's scale,
+ *   rounded to nearest), so the result equals mla_absorb_q / mla_out_up given that bf16 weight.
+ *   bf16 activations and outputs, DeepSeek dimensions only.  Asynchronous on `stream`.
+ */
+mla_status mla_absorb_q_fp8(mla_dims dims, int32_t B, const void* q_nope, int64_t ldq, const void* w_fp8,
+                            const float* w_scale, void* q_tilde, int32_t* dev_err, void* stream);
+mla_status mla_out_up_fp8(mla_dims dims, int32_t B, const void* ctx, const void* w_fp8, const float* w_scale,
+                          void* out, int32_t* dev_err, void* stream);
+
+/*
  * mla_prefill_workspace_size - bytes of scratch mla_prefill_naive needs: the expanded
  * [B, S, n_h, d_h + d_v] keys/values in the input dtype.
  */
@@ -237,6 +253,29 @@ mla_status mla_cache_append(mla_dims dims, mla_dtype dtype, int32_t B,
  */
 mla_status mla_check_topk(int32_t B, const int32_t* topk_idx, int32_t topk, const int32_t* lengths, int32_t n_max,
                           int32_t* dev_err, void* stream);
+
+/*
+ * mla_prefill_sparse_workspace_size - bytes of scratch mla_prefill_sparse needs: the expansion of
+ * mla_prefill_workspace_size plus the per-row selection bitmaps and per-query-tile key-tile lists.
+ */
+size_t mla_prefill_sparse_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S);
+
+/*
+ * mla_prefill_sparse - the V3.2 sparse prefill ("Value up-projection", MHA-prefill excerpt: a -inf
+ * row with 0 scattered at each query row's top-k positions, plus the causal mask, added to the
+ * scores): as mla_prefill_naive with causal = 1, except that query row s attends only the
+ * positions t <= s listed in its row of topk_idx (a set: repeats count once).
+ *   topk_idx  DEVICE int32 [B, S, topk] contiguous; an index outside [0, S) sets MLA_ERR_INDEX and
+ *             is ignored; indices past the row (t > s) are removed by the causal mask
+ *   a row whose set holds no t <= s has no softmax: it is written as zeros and MLA_ERR_INDEX is set
+ *   bf16 DeepSeek dimensions only (MLA_ERR_UNSUPPORTED otherwise).
+ * Asynchronous on `stream`.
+ */
+mla_status mla_prefill_sparse(mla_dims dims, mla_dtype dtype, int32_t B, int32_t S,
+                              const void* q, const void* c_kv, int64_t ckv_rstride,
+                              const void* k_r, int64_t kr_rstride, const void* w_kv_b,
+                              float scale, const int32_t* topk_idx, int32_t topk, void* out,
+                              void* workspace, size_t ws_bytes, int32_t* dev_err, void* stream);
 
 /* Zero the device flag (asynchronous on `stream`). */
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream);
