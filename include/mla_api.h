@@ -13,6 +13,10 @@
  *   mla_cache_append   the new token's latent (RMSNorm) and rotary key (RoPE) into the caches
  *                                                                    ("Key-value down-projection", mla-kv
  *                                                                     excerpt; "Key-value latent RMSNorm")
+ *   mla_prefill_sparse the V3.2 prefill: each query row attends its top-k positions t <= s
+ *                                                                    ("Value up-projection", MHA-prefill excerpt)
+ *   mla_absorb_q_fp8, mla_out_up_fp8  the projections with an FP8 wkv_b and its 128 x 128 block scales
+ *                                                                    ("Key-value down-projection", linear excerpt)
  * plus one opt-in check of the sparse decode's precondition:
  *   mla_check_topk     top-k indices in range and distinct per sequence (the mask is a set)
  *
