@@ -110,6 +110,20 @@ def test_host_validation_codes(L):
                               FAKE, 8 * 64, 64, FAKE, 8 * 15, 15, None, None) == 1   # odd rotary width
     assert L.mla_cache_append(tiny, bf, 1, FAKE, 80, None, 1e-6, 1e4, FAKE, 8,
                               FAKE, 8 * 64, 64, FAKE, 8 * 16, 16, None, None) == 2   # bf16 outside DeepSeek dims
+    # sparse prefill and FP8 projections
+    assert L.mla_prefill_sparse(DS, f32, 1, 16, FAKE, FAKE, 576, FAKE, 576, FAKE, 0.07, FAKE, 8, FAKE, FAKE,
+                                1 << 30, None, None) == 2                     # bf16 only
+    assert L.mla_prefill_sparse(DS, bf, 1, 16, FAKE, FAKE, 576, FAKE, 576, FAKE, 0.07, None, 8, FAKE, FAKE,
+                                1 << 30, None, None) == 1                     # no top-k array
+    assert L.mla_prefill_sparse(DS, bf, 1, 16, FAKE, FAKE, 576, FAKE, 576, FAKE, 0.07, FAKE, 8, FAKE, None,
+                                0, None, None) == 6                           # no workspace
+    assert L.mla_prefill_sparse_workspace_size(DS, bf, 2, 2048) > L.mla_prefill_workspace_size(DS, bf, 2, 2048)
+    assert L.mla_prefill_sparse_workspace_size(DS, f32, 2, 2048) == 0
+    assert L.mla_absorb_q_fp8(DS, 1, FAKE, 128, FAKE, None, FAKE, None, None) == 1   # no scales
+    assert L.mla_absorb_q_fp8(DS, 1, FAKE, 100, FAKE, FAKE, FAKE, None, None) == 1   # ldq below d_h
+    assert L.mla_absorb_q_fp8(tiny, 1, FAKE, 32, FAKE, FAKE, FAKE, None, None) == 2  # not the DeepSeek dims
+    assert L.mla_out_up_fp8(DS, 0, FAKE, FAKE, FAKE, FAKE, None, None) == 1
+    assert L.mla_out_up_fp8(DS, 1, FAKE, FAKE + 8, FAKE, FAKE, None, None) == 1     # misaligned weight
     # top-k validation
     assert L.mla_check_topk(0, FAKE, 8, None, 64, FAKE, None) == 1
     assert L.mla_check_topk(2, None, 8, None, 64, FAKE, None) == 1
