@@ -230,6 +230,58 @@ def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append
                              "note": "a few KB per call: bound by launch latency, not by HBM"}
         del cache
         torch.cuda.empty_cache()
+    if "fp8proj" in which:
+        # the two projections of the decode workload with an e4m3 wkv_b and 128 x 128 block scales
+        cfg = V3_DECODE
+        rng = np.random.default_rng(cfg.seed + 200)
+        w = torch.from_numpy(rng.standard_normal((cfg.n_h * (cfg.d_h + cfg.d_v), cfg.d_c), dtype=np.float32) * 0.02)
+        amax = w.reshape(w.shape[0] // 128, 128, cfg.d_c // 128, 128).abs().amax(dim=(1, 3)).clamp_min(1e-12)
+        scale = (amax / 448.0).float()
+        wq = (w / scale.repeat_interleave(128, 0).repeat_interleave(128, 1)).to(torch.float8_e4m3fn).to(dev)
+        scale = scale.to(dev)
+        q_nope = torch.from_numpy(rng.standard_normal((cfg.B, cfg.n_h, cfg.d_h), dtype=np.float32)).to(
+            torch.bfloat16).to(dev)
+        ctx = torch.from_numpy(rng.standard_normal((cfg.B, cfg.n_h, cfg.d_c), dtype=np.float32) * 0.05).to(
+            torch.bfloat16).to(dev)
+        qt = torch.empty((cfg.B, cfg.n_h, cfg.d_c), dtype=torch.bfloat16, device=dev)
+        o = torch.empty((cfg.B, cfg.n_h, cfg.d_v), dtype=torch.bfloat16, device=dev)
+        half_w = cfg.n_h * cfg.d_h * cfg.d_c  # fp8 bytes of one projection's weight half
+        for name, fn, nbytes in (
+                ("absorb_q_fp8", lambda: api.mla_absorb_q_fp8(cfg.dims, q_nope, wq, scale, q_tilde=qt, stream=stream),
+                 half_w + cfg.B * cfg.n_h * (cfg.d_h + cfg.d_c) * 2),
+                ("out_up_fp8", lambda: api.mla_out_up_fp8(cfg.dims, ctx, wq, scale, out=o, stream=stream),
+                 half_w + cfg.B * cfg.n_h * (cfg.d_c + cfg.d_v) * 2)):
+            ms = timed(fn)
+            gbs = nbytes / (ms * 1e-3) / 1e9
+            out[name + "_b32"] = {"call": "mla_" + name, "ms": ms, "algorithmic_bytes": nbytes, "achieved_GBs": gbs,
+                                  "hbm_frac": gbs / peaks["hbm_gbs"]}
+        del wq
+        torch.cuda.empty_cache()
+    if "sparse_prefill" in which:
+        # a V3.2-style sparse prefill: B=1, S=8192, each row's 2048 selected positions (itself plus
+        # 2047 drawn over the sequence; the causal mask removes the later ones)
+        cfg = PREFILL.with_(B=1, n_max=8192)
+        p = make_prefill_inputs(cfg)
+        S, k = cfg.n_max, 2048
+        rng = np.random.default_rng(cfg.seed + 300)
+        topk = np.empty((1, S, k), dtype=np.int32)
+        for s_ in range(S):
+            topk[0, s_, 0] = s_
+            topk[0, s_, 1:] = rng.choice(S, k - 1, replace=False)
+        visible = sum(len({t for t in topk[0, s_].tolist() if t <= s_}) for s_ in range(S))
+        q, c_kv, k_r, w = p["q"].to(dev), p["c_kv"].to(dev), p["k_r"].to(dev), p["w_kv_b"].to(dev)
+        tk = torch.from_numpy(topk).to(dev)
+        o = torch.empty((1, S, cfg.n_h, cfg.d_v), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((int(api.lib().mla_prefill_sparse_workspace_size(api._dims(cfg.dims), 1, 1, S)),),
+                         dtype=torch.uint8, device=dev)
+        ms = timed(lambda: api.mla_prefill_sparse(cfg.dims, q, c_kv, k_r, w, cfg.scale, tk, out=o, workspace=ws,
+                                                  stream=stream))
+        flops = 2 * S * cfg.n_h * (cfg.d_h + cfg.d_v) * cfg.d_c + 2 * cfg.n_h * visible * ((cfg.d_h + cfg.d_r) + cfg.d_v)
+        tf = flops / (ms * 1e-3) / 1e12
+        out["sparse_prefill_b1_s8192_k2048"] = {"call": "mla_prefill_sparse", "ms": ms, "visible_pairs": visible,
+                                                "flops": flops, "tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"]}
+        del q, c_kv, k_r, w, tk, o, ws
+        torch.cuda.empty_cache()
     if "prefill" not in which:
         return out
     cfg = PREFILL
@@ -411,7 +463,7 @@ def main():
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the timings of the ragged, top-k and prefill workloads")
-    ap.add_argument("--only", choices=["ragged", "sparse", "prefill", "append"],
+    ap.add_argument("--only", choices=["ragged", "sparse", "prefill", "append", "fp8proj", "sparse_prefill"],
                     help="time only this secondary workload (--steps launches after 3 warm-up ones) and print "
                          "its entry; a small command for profilers, not a bench line")
     args = ap.parse_args()
