@@ -47,7 +47,7 @@ def test_sparse_prefill_against_oracle(dev, S, k):
         check_close(out[b][:, heads], want, torch.bfloat16, f"sparse prefill S={S} b={b}")
 
 
-def test_every_position_selected_equals_dense(dev):
+def test_every_position_selected_matches_dense(dev):
     cfg = PREFILL.with_(B=1, n_max=384)
     p = make_prefill_inputs(cfg)
     S = cfg.n_max
@@ -56,4 +56,7 @@ def test_every_position_selected_equals_dense(dev):
     sp = api.mla_prefill_sparse(*args, torch.from_numpy(topk).cuda())
     dense = api.mla_prefill_naive(*args)
     torch.cuda.synchronize()
-    assert torch.equal(sp, dense)
+    # the same arithmetic in the same order; the two kernel instantiations may still contract a
+    # multiply-add differently, so allow one bf16 ulp
+    diff = (sp.float() - dense.float()).abs()
+    assert bool((diff <= dense.float().abs() * 2.0 ** -7 + 1e-6).all()), float(diff.max())
