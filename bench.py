@@ -35,8 +35,8 @@ METRIC = "MLA absorbed-decode tokens/s and % of roofline (B=32, N=4096, 128 head
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch on this workload,
-# from the ncu capture summarised in profiles/decode_kernel_v3_b32_n4096.md, valid only for the
-# kernel source it was taken on (sha256 prefix of csrc/decode_sm100.cu).
+# from one ncu capture of the decode kernel, valid only for the kernel source it was taken on
+# (sha256 prefix of csrc/decode_sm100.cu).
 DECODE_TRAFFIC = {"bytes": 155_848_960 + 7_039_232, "source_sha256": "af96b1671f600577"}
 
 
