@@ -55,6 +55,7 @@ SIGNATURES = {
     "mla_prefill_sparse_workspace_size": (c_sz, [MLADims, c_i32, c_i32, c_i32]),
     "mla_prefill_sparse": (c_i32, [MLADims, c_i32, c_i32, c_i32, c_vp, c_vp, c_i64, c_vp, c_i64, c_vp,
                                    c_f32, c_vp, c_i32, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "mla_selftest_wait_timeout": (c_i32, [ctypes.c_uint64, c_vp, c_vp]),
     "mla_clear_device_error": (c_i32, [c_vp, c_vp]),
     "mla_get_device_error": (c_i32, [c_vp, c_i32p]),
 }

@@ -11,6 +11,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "sm100_ptx.cuh"
 
 namespace mla {
 namespace {
@@ -115,6 +116,26 @@ __global__ void __launch_bounds__(kCheckThreads) check_topk_kernel(const int32_t
 }
 
 }  // namespace
+
+// The bounded wait every kernel uses, made to run out: an mbarrier expecting one arrival that never
+// comes.  The wait gives up after limit_ns of global time and the flag records MLA_ERR_TIMEOUT.
+__global__ void __launch_bounds__(32) wait_timeout_kernel(uint64_t limit_ns, int32_t* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(sm100::smem_u32(&bar), 1);
+    abort_flag = 0;
+    sm100::fence_mbar_init();
+  }
+  __syncwarp();
+  const bool done = sm100::mbar_wait(sm100::smem_u32(&bar), 0, &abort_flag, limit_ns);
+  if (threadIdx.x == 0 && !done) raise_error(err, MLA_ERR_TIMEOUT);
+}
+
+cudaError_t wait_timeout_launch(uint64_t limit_ns, int32_t* err, cudaStream_t st) {
+  wait_timeout_kernel<<<1, 32, 0, st>>>(limit_ns, err);
+  return cudaGetLastError();
+}
 
 size_t check_topk_smem_bytes(int n_max) { return (size_t)((n_max + 31) / 32) * sizeof(uint32_t); }
 

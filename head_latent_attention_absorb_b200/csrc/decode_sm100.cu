@@ -1642,8 +1642,7 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
 // ------------------------------------------------------------------------------------------
 // Some callers cannot allocate device memory when they run a decode: a plugin or engine host
 // whose enqueue callback may not call cudaMalloc (it would synchronise or break the host's memory
-// budget), code issuing work while a stream is being captured into a CUDA graph, or a caller that
-// only holds pointers handed to it by someone else.  For them the split-KV scratch lives in this
+// budget), or a caller that only holds pointers handed to it by someone else.  For them the split-KV scratch lives in this
 // file-scope array, which every GPU that loads the library holds until the process exits.
 // Sized for 74 clusters (one CTA pair per two SMs of a 148-SM B200) and up to 4096 sequences:
 // 74 x 2 partial slots of 128 heads x 512 bf16 features, their (m, l) pairs and ready flags, and

@@ -29,6 +29,7 @@ cudaError_t cache_append_launch(const AppendArgs& a, cudaStream_t st);
 
 // ---- top-k index validation (range and distinctness per sequence) --------------------------
 size_t check_topk_smem_bytes(int n_max);
+cudaError_t wait_timeout_launch(uint64_t limit_ns, int32_t* err, cudaStream_t st);
 cudaError_t check_topk_launch(int B, const int32_t* idx, int topk, const int32_t* lengths, int n_max, int32_t* err,
                               cudaStream_t st);
 

@@ -387,6 +387,14 @@ mla_status mla_prefill_sparse(mla_dims dims, mla_dtype dtype, int32_t B, int32_t
   return cuda_status(e, "mla_prefill_sparse launch");
 }
 
+mla_status mla_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  if (!dev_err) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (limit_ns < 1000 || limit_ns > 1000000000ull) return fail(MLA_ERR_INVALID_ARG, "limit_ns outside [1 us, 1 s]");
+  return cuda_status(mla::wait_timeout_launch(limit_ns, dev_err, static_cast<cudaStream_t>(stream)),
+                     "mla_selftest_wait_timeout launch");
+}
+
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream) {
   g_msg[0] = 0;
   if (!dev_err) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");

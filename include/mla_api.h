@@ -143,9 +143,10 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
 /*
  * mla_decode_absorb_static - mla_decode_absorb for the bf16 dense decode (no top-k) WITHOUT a
  * caller-supplied workspace.  The pages have no counterpart: this is a deployment convenience.
- *   For callers that cannot allocate device memory around a decode call: a plugin / engine host
- *   whose enqueue path may not call cudaMalloc, code issuing work while a stream is being captured
- *   into a CUDA graph, or a caller that only holds pointers handed to it.  The split-KV scratch is
+ *   For callers that cannot allocate device memory around a decode call: a plugin or engine host
+ *   whose enqueue path may not call cudaMalloc (an allocation there can synchronise the device or
+ *   break the host's own memory budget), or a caller that only holds pointers handed to it by
+ *   someone else and owns no allocator.  The split-KV scratch is
  *   a file-scope device array of 19,769,920 bytes (about 18.9 MiB: 74 clusters x 2 bf16 partial
  *   slots), held by every GPU that loads the library until the process exits.
  *   Arguments and results are those of mla_decode_absorb with topk_idx = NULL and without
@@ -280,6 +281,14 @@ mla_status mla_prefill_sparse(mla_dims dims, mla_dtype dtype, int32_t B, int32_t
                               const void* k_r, int64_t kr_rstride, const void* w_kv_b,
                               float scale, const int32_t* topk_idx, int32_t topk, void* out,
                               void* workspace, size_t ws_bytes, int32_t* dev_err, void* stream);
+
+/*
+ * mla_selftest_wait_timeout - failure detection without a fault: one CTA waits on an mbarrier that
+ * nothing arrives on, with the bounded wait every kernel of the library uses; after limit_ns
+ * (1 us .. 1 s) of global time it gives up and sets MLA_ERR_TIMEOUT in dev_err.  The context stays
+ * usable.  Asynchronous on `stream`.
+ */
+mla_status mla_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_err, void* stream);
 
 /* Zero the device flag (asynchronous on `stream`). */
 mla_status mla_clear_device_error(int32_t* dev_err, void* stream);
