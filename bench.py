@@ -165,11 +165,13 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append")):
+def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append", "fp8proj", "sparse_prefill",
+                                          "multi")):
     """The other workloads of the hot path, each timed on its own with CUDA events (L2 flushed
     before every launch): the ragged long-context decode, the V3.2 top-k decode, the naive causal
-    prefill and the cache append of one new token per sequence in front of the decode.  Reported
-    beside the headline line; algorithmic bytes / FLOPs as for the headline."""
+    prefill, the cache append of one new token per sequence in front of the decode, the two
+    projections with an FP8 wkv_b, and a V3.2 sparse prefill.  Reported beside the headline line;
+    algorithmic bytes / FLOPs as for the headline."""
     from head_latent_attention_absorb_b200 import api
     from head_latent_attention_absorb_b200.configs import PREFILL, RAGGED_LONG, SPARSE_V32
     from head_latent_attention_absorb_b200.inputs import make_prefill_inputs
@@ -229,6 +231,37 @@ def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append
                              "algorithmic_bytes": nbytes, "achieved_GBs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
                              "note": "a few KB per call: bound by launch latency, not by HBM"}
         del cache
+        torch.cuda.empty_cache()
+    if "multi" in which:
+        # two new tokens per sequence (e.g. a speculative token) on the decode workload's cache: each
+        # token attends its visible rows; algorithmic bytes count the cache once
+        cfg, T = V3_DECODE, 2
+        x = make_decode_inputs(cfg)
+        cache = x["cache"].to(dev)
+        c_kv, k_r = cache[..., :cfg.d_c], cache[..., cfg.d_c:]
+        rng = np.random.default_rng(cfg.seed + 400)
+        qt = torch.from_numpy(rng.standard_normal((cfg.B, T, cfg.n_h, cfg.d_c), dtype=np.float32) * 0.2).to(
+            torch.bfloat16).to(dev)
+        qp = torch.from_numpy(rng.standard_normal((cfg.B, T, cfg.n_h, cfg.d_r), dtype=np.float32)).to(
+            torch.bfloat16).to(dev)
+        lengths = x["lengths"].to(dev)
+        ctx = torch.empty((cfg.B, T, cfg.n_h, cfg.d_c), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((api.mla_decode_workspace_size(cfg.dims, torch.bfloat16, cfg.B * T, cfg.n_max),),
+                         dtype=torch.uint8, device=dev)
+        ms = timed(lambda: api.mla_decode_absorb_multi(cfg.dims, qt, qp, c_kv, k_r, lengths, cfg.scale, ctx=ctx,
+                                                       workspace=ws, stream=stream))
+        lens = x["lengths"].to(torch.int64)
+        keys = int(sum(int(L) - T + 1 + s_ for L in lens for s_ in range(T)))
+        nbytes = int(lens.sum()) * (cfg.d_c + cfg.d_r) * 2 + cfg.B * T * cfg.n_h * (2 * cfg.d_c + cfg.d_r) * 2
+        flops = 2 * keys * cfg.n_h * (2 * cfg.d_c + cfg.d_r)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tf = flops / (ms * 1e-3) / 1e12
+        out["multi_b32_t2_n4096"] = {"call": "mla_decode_absorb_multi", "ms": ms, "tokens_per_s": cfg.B * T / (ms * 1e-3),
+                                     "algorithmic_bytes": nbytes, "achieved_GBs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                                     "flops": flops, "tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"],
+                                     "roofline_frac": max(nbytes / (peaks["hbm_gbs"] * 1e9),
+                                                          flops / (peaks["bf16_tflops"] * 1e12)) / (ms * 1e-3)}
+        del x, cache, c_kv, k_r, ws
         torch.cuda.empty_cache()
     if "fp8proj" in which:
         # the two projections of the decode workload with an e4m3 wkv_b and 128 x 128 block scales
@@ -462,8 +495,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--ref-budget-s", type=float, default=120.0)
     ap.add_argument("--no-secondary", action="store_true",
-                    help="skip the timings of the ragged, top-k and prefill workloads")
-    ap.add_argument("--only", choices=["ragged", "sparse", "prefill", "append", "fp8proj", "sparse_prefill"],
+                    help="skip the timings of the secondary workloads (ragged, top-k, prefill, cache append, "
+                         "FP8 projections, sparse prefill)")
+    ap.add_argument("--only", choices=["ragged", "sparse", "prefill", "append", "fp8proj", "sparse_prefill", "multi"],
                     help="time only this secondary workload (--steps launches after 3 warm-up ones) and print "
                          "its entry; a small command for profilers, not a bench line")
     args = ap.parse_args()

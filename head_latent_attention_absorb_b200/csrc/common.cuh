@@ -39,6 +39,7 @@ __device__ __forceinline__ void raise_error(int32_t* flag, int32_t code) {
 // Validated arguments of one decode call (pointers already checked on the host).
 struct DecodeArgs {
   int n_h, d_c, d_r, B, n_max, topk;
+  int T = 1;  // new tokens per cache sequence: B query groups over B / T cache sequences
   const void* q_tilde; int64_t ldqt;
   const void* q_pe;    int64_t ldqp;
   const void* c_kv;    int64_t ckv_b, ckv_r;

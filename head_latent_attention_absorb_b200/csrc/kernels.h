@@ -35,6 +35,8 @@ cudaError_t check_topk_launch(int B, const int32_t* idx, int topk, const int32_t
 
 // ---- tcgen05 kernels (bf16, DeepSeek-V3 dimensions) ------------------------------------------
 size_t decode_tc_workspace(int B);
+size_t decode_pair_workspace(int B);
+cudaError_t decode_pair_launch(const DecodeArgs& a, void* ws, cudaStream_t st);
 cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st);
 cudaError_t absorb_q_tc_launch(int B, const void* q_nope, int64_t ldq, const void* w, void* q_tilde, cudaStream_t st);
 cudaError_t out_up_tc_launch(int B, const void* ctx, const void* w, void* out, cudaStream_t st);

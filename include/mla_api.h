@@ -141,6 +141,30 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
                              void* workspace, size_t ws_bytes, int32_t* dev_err, void* stream);
 
 /*
+ * mla_decode_absorb_multi - mla_decode_absorb for T new tokens per sequence ("DeepSeek-V3.2-Exp -
+ * Absorb key weights", decode excerpt: the queries are [batch, s, heads, features] with s = T, e.g.
+ * speculative tokens).  The T tokens of sequence b are the last T of its lengths[b] cached rows;
+ * token s (0-based) attends rows t <= lengths[b] - T + s, the causal rule of the prefill excerpt
+ * ("Value up-projection", MHA-prefill excerpt), so T = 1 is mla_decode_absorb.
+ *   q_tilde, q_pe, ctx_out, lse_out  [B * T, n_h, .] with row (b * T + s, h), strides as in
+ *                                    mla_decode_absorb (query rows (b * T + s) * n_h + h)
+ *   c_kv, k_r                        [B, n_max, .] caches as in mla_decode_absorb
+ *   lengths                          DEVICE int32 [B], each in [T, n_max]; a shorter or longer one
+ *                                    sets MLA_ERR_LENGTH in dev_err and its tokens get ctx = 0,
+ *                                    lse = -inf
+ *   workspace                        mla_decode_workspace_size(dims, dtype, B * T, n_max, 0) bytes
+ * bf16 DeepSeek dimensions only, no top-k set for T > 1 (MLA_ERR_UNSUPPORTED).  Each token runs as
+ * its own query group over the shared cache rows of its sequence.  Asynchronous on `stream`.
+ */
+mla_status mla_decode_absorb_multi(mla_dims dims, mla_dtype dtype, int32_t B, int32_t T,
+                                   const void* q_tilde, int64_t ldqt, const void* q_pe, int64_t ldqp,
+                                   const void* c_kv, int64_t ckv_bstride, int64_t ckv_rstride,
+                                   const void* k_r, int64_t kr_bstride, int64_t kr_rstride,
+                                   int32_t n_max, const int32_t* lengths, float scale, void* ctx_out,
+                                   float* lse_out, void* workspace, size_t ws_bytes, int32_t* dev_err,
+                                   void* stream);
+
+/*
  * mla_decode_absorb_static - mla_decode_absorb for the bf16 dense decode (no top-k) WITHOUT a
  * caller-supplied workspace.  The pages have no counterpart: this is a deployment convenience.
  *   For callers that cannot allocate device memory around a decode call: a plugin or engine host
