@@ -5,6 +5,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+#include <stdlib.h>
 
 #include "mla_api.h"
 
@@ -34,6 +35,18 @@ __device__ __forceinline__ float warp_max(float v) {
 // First error wins: a later error never overwrites an earlier one.
 __device__ __forceinline__ void raise_error(int32_t* flag, int32_t code) {
   if (flag != nullptr) atomicCAS(flag, 0, code);
+}
+
+// Whether a persistent decode launch may use the sliced merge, in which every cluster holding a
+// piece of a sequence waits for all the others' partials.  That wait needs every cluster of the
+// launch resident at once.  The launcher passes `one_wave` = the occupancy query confirmed that the
+// whole grid fits on the GPU in one wave; MLA_DECODE_SLICED_MERGE=0 in the environment turns the
+// sliced merge off as well, for GPUs whose SMs another context may hold for the length of a launch
+// (MPS clients, another process's long-running kernel).  Without it the last cluster to arrive
+// merges every partial, which waits only on clusters that have already run.
+inline bool sliced_merge_allowed(bool one_wave) {
+  const char* e = getenv("MLA_DECODE_SLICED_MERGE");
+  return one_wave && !(e != nullptr && e[0] == '0' && e[1] == '\0');
 }
 
 // Validated arguments of one decode call (pointers already checked on the host).

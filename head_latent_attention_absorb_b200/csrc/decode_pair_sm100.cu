@@ -95,6 +95,7 @@ struct Params {
   int64_t ldqt;
   const int32_t* lengths;       // [B / T] cached rows per cache sequence
   int B, n_max, n_clusters;     // B query rows groups (pseudo-sequences): T per cache sequence
+  int slice_above;              // more partials than this: the sliced merge (needs every cluster resident)
   int T;                        // new tokens per cache sequence (1 for the one-token decode)
   float scale_log2;
   __nv_bfloat16* ctx;
@@ -638,12 +639,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (i == end - 1 && !whole) {
             // The segment's last tile is under way: count this cluster's arrival for the sequence now
             // (an atomic costs a microsecond when HBM is saturated; here it overlaps the tile's
-            // softmax and P.V instead of delaying the epilogue).  With up to kMergeLastMax partials the
-            // last cluster to arrive merges them all, so it must know; with more, every cluster merges
-            // a slice and counts its arrival afterwards.  The epilogue of the previous segment has
+            // softmax and P.V instead of delaying the epilogue).  With up to p.slice_above partials
+            // (kMergeLastMax when the whole grid is resident, else any number) the last cluster to
+            // arrive merges them all, so it must know; with more, every cluster merges a slice and
+            // counts its arrival afterwards.  The epilogue of the previous segment has
             // finished reading the slot list (this segment's first score MMA needed its query).
             const int ns = list_slots(p, sm, base, tiles_of(len));
-            sm.is_last = ns > kMergeLastMax ? 0 : (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0);
+            sm.is_last = ns > p.slice_above ? 0 : (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0);
             mbar_arrive(smem_u32(&sm.last_bar));
           }
         }
@@ -1046,7 +1048,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             st_release_gpu(p.ws_ready + 2 * (int64_t)own + rank, p.epoch);
           }
         }
-        if (sm.nslots > kMergeLastMax) {
+        if (sm.nslots > p.slice_above) {
           // ---- sliced merge: every slot's partial is published; this CTA merges heads [h_lo, h_hi)
           // of its 64, one head per warp and two 16-byte chunks per lane (a warp reads and writes
           // 512 contiguous bytes per step), summing the slots in slot order.  The last cluster to
@@ -1127,10 +1129,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          // In the range's last segment the other partials are loaded by TMA into the free stage area
-          // (partial k of the others at k x 64 KB, in the same swizzled boxes as the staging), and
-          // with one other partial the output is staged behind it and stored by TMA.
-          const bool bulk = last_seg;
+          // In the range's last segment up to three other partials are loaded by TMA into the free
+          // stage area (partial k of the others at k x 64 KB, in the same swizzled boxes as the
+          // staging), and with one other partial the output is staged behind it and stored by TMA.
+          // More partials (the sliced merge turned off) are read through L2.
+          const bool bulk = last_seg && ns <= kMergeLastMax;
           const bool staged = last_seg && ns == 2;
           // (m, l) of the k-th other partial: in shared memory after the bulk loads, else in L2
           const float2* ml_smem = reinterpret_cast<const float2*>(smem + 196608);
@@ -1166,7 +1169,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           // its reads cost a round trip to L2.)
           float M = -INFINITY;
           for (int s2 = 0; s2 < ns; ++s2) M = fmaxf(M, ml_of(s2).x);
-          float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f;
+          float w0 = 0.f, w1 = 0.f, w2 = 0.f, w3 = 0.f, inv = 0.f;
           float L;
           if (ns == 2) {
             // two terms, each rounded once, added once: the same sum in either arrival order
@@ -1181,8 +1184,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               const float2 ml = ml_of(s2);
               L += ml.y * ex2f_approx(ml.x - M);
             }
-            const float inv = 1.f / L;
-            for (int s2 = 0; s2 < ns; ++s2) {
+            inv = 1.f / L;
+            for (int s2 = 0; s2 < ns && s2 < 4; ++s2) {
               const float2 ml = ml_of(s2);
               const float w = ml.y * ex2f_approx(ml.x - M) * inv;
               w0 = s2 == 0 ? w : w0;
@@ -1244,7 +1247,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int kb2 = 0;
             for (int s2 = 0; s2 < ns; ++s2) {
               const int sl = sm.slots[s2];
-              const float w = s2 == 0 ? w0 : (s2 == 1 ? w1 : (s2 == 2 ? w2 : w3));
+              float w = s2 == 0 ? w0 : (s2 == 1 ? w1 : (s2 == 2 ? w2 : w3));
+              if (s2 >= 4) {  // beyond four slots the weight is formed here, from (m, l) in L2
+                const float2 ml = ml_of(s2);
+                w = ml.y * ex2f_approx(ml.x - M) * inv;
+              }
               if (sl == own) {
                 if (ns == 2) {
 #pragma unroll
@@ -1345,14 +1352,21 @@ int max_clusters() {
   return n > 0 ? n : 1;
 }
 
-// Clusters that can be resident at once, so that the grid is exactly one wave.  Cached per device.
-int num_clusters() {
-  static int cache[64] = {0};
+// Clusters of the persistent grid: as many CTA pairs as can be resident at once, so that the grid is
+// exactly one wave.  `one_wave` records whether the occupancy query confirmed that (when it fails the
+// grid takes the upper bound and the sliced merge, which needs every cluster resident, is not used).
+// Cached per device.
+struct Wave {
+  int clusters;
+  bool one_wave;
+};
+Wave grid_wave() {
+  static Wave cache[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  if (dev >= 0 && dev < 64 && cache[dev].clusters > 0) return cache[dev];
   const int upper = max_clusters();
-  int n = upper;
+  Wave w{upper, false};
   if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes()) ==
       cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -1360,12 +1374,14 @@ int num_clusters() {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem_bytes();
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, decode_kernel, &cfg) == cudaSuccess && active > 0 && active < n)
-      n = active;
+    if (cudaOccupancyMaxActiveClusters(&active, decode_kernel, &cfg) == cudaSuccess && active > 0) {
+      w.clusters = active < upper ? active : upper;
+      w.one_wave = true;
+    }
   }
   cudaGetLastError();
-  if (dev >= 0 && dev < 64) cache[dev] = n;
-  return n;
+  if (dev >= 0 && dev < 64) cache[dev] = w;
+  return w;
 }
 
 }  // namespace decode_pair
@@ -1374,7 +1390,8 @@ size_t decode_pair_workspace(int B) { return decode_pair::ws_bytes(decode_pair::
 
 cudaError_t decode_pair_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   using namespace decode_pair;
-  const int nc = num_clusters();
+  const Wave wave = grid_wave();
+  const int nc = wave.clusters;
   Params p;
   memset(&p, 0, sizeof(p));
   const int T = a.T > 0 ? a.T : 1;
@@ -1406,6 +1423,7 @@ cudaError_t decode_pair_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   p.T = T;
   p.n_max = a.n_max;
   p.n_clusters = nc;
+  p.slice_above = sliced_merge_allowed(wave.one_wave) ? kMergeLastMax : 0x7fffffff;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.ctx = static_cast<__nv_bfloat16*>(a.ctx);
   p.lse = a.lse;

@@ -91,6 +91,7 @@ struct Params {
   int64_t ldqp;
   const int32_t* lengths;
   int B, n_max, n_clusters;
+  int slice_above;  // more partials than this: the sliced merge (needs every cluster resident at once)
   float scale_log2;
   __nv_bfloat16* ctx;
   float* lse;
@@ -1038,9 +1039,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int own = 2 * cl + (first_seg ? 0 : 1);
         if (sw == 0 && lane == 0) {
           const int ns = list_slots(p, sm, base, tiles_of(len));
-          // up to kMergeLastMax partials the last cluster to arrive merges them all; with more, every
-          // cluster publishes and then merges its own slice of the heads
-          sm.is_last = ns > kMergeLastMax ? 0 : (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0);
+          // up to p.slice_above partials (kMergeLastMax when the whole grid is resident, else any
+          // number) the last cluster to arrive merges them all; with more, every cluster publishes and
+          // then merges its own slice of the heads
+          sm.is_last = ns > p.slice_above ? 0 : (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0);
           mbar_arrive(smem_u32(&sm.last_bar));
         }
         if (!wait_or_fail(smem_u32(&sm.last_bar), npart & 1u, false)) break;
@@ -1081,7 +1083,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           ++npub;
         }
-        if (sm.nslots > kMergeLastMax) {
+        if (sm.nslots > p.slice_above) {
           // ---- sliced merge: every slot's partial is published (lane 0 of each warp polls the flags,
           // this cluster's own included); this CTA merges heads [h_lo, h_hi) of its latent half, one
           // head per warp and one 16-byte chunk per lane, summing the slots in slot order.  The last
@@ -1551,15 +1553,21 @@ int max_clusters() {
   return n > 0 ? n : 1;
 }
 
-// Clusters that can be resident at once (GPCs with an odd number of free SMs cannot host a full
-// pair), so that the persistent grid is exactly one wave.  Cached per device.
-int num_clusters() {
-  static int cache[64] = {0};
+// Clusters of the persistent grid: as many CTA pairs as can be resident at once (GPCs with an odd
+// number of free SMs cannot host a full pair), so that the grid is exactly one wave.  `one_wave`
+// records whether the occupancy query confirmed that (when it fails the grid takes the upper bound
+// and the sliced merge, which needs every cluster resident, is not used).  Cached per device.
+struct Wave {
+  int clusters;
+  bool one_wave;
+};
+Wave grid_wave() {
+  static Wave cache[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  if (dev >= 0 && dev < 64 && cache[dev].clusters > 0) return cache[dev];
   const int upper = max_clusters();
-  int n = upper;
+  Wave w{upper, false};
   if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes()) ==
       cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
@@ -1567,12 +1575,14 @@ int num_clusters() {
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem_bytes();
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, decode_kernel, &cfg) == cudaSuccess && active > 0 && active < n)
-      n = active;
+    if (cudaOccupancyMaxActiveClusters(&active, decode_kernel, &cfg) == cudaSuccess && active > 0) {
+      w.clusters = active < upper ? active : upper;
+      w.one_wave = true;
+    }
   }
-  cudaGetLastError();  // a failed query leaves no sticky state; keep the upper bound
-  if (dev >= 0 && dev < 64) cache[dev] = n;
-  return n;
+  cudaGetLastError();  // a failed query leaves no sticky state
+  if (dev >= 0 && dev < 64) cache[dev] = w;
+  return w;
 }
 
 }  // namespace decode_tc
@@ -1581,7 +1591,8 @@ size_t decode_tc_workspace(int B) { return decode_tc::ws_bytes(decode_tc::max_cl
 
 cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   using namespace decode_tc;
-  const int nc = num_clusters();
+  const Wave wave = grid_wave();
+  const int nc = wave.clusters;
   Params p;
   memset(&p, 0, sizeof(p));
   const uint64_t bstride_c = a.B > 1 ? (uint64_t)a.ckv_b * 2 : (uint64_t)a.n_max * a.ckv_r * 2;
@@ -1617,6 +1628,7 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   p.B = a.B;
   p.n_max = a.n_max;
   p.n_clusters = nc;
+  p.slice_above = sliced_merge_allowed(wave.one_wave) ? kMergeLastMax : 0x7fffffff;
   p.scale_log2 = a.scale * 1.4426950408889634f;
   p.ctx = static_cast<__nv_bfloat16*>(a.ctx);
   p.lse = a.lse;

@@ -130,6 +130,13 @@ int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32
  *            contents need no initialisation and are garbage afterwards
  *   dev_err  NULL or a device int32 flag; MLA_ERR_LENGTH / MLA_ERR_INDEX are stored there
  * Asynchronous on `stream`.
+ * Residency: the kernel is one persistent wave of CTA pairs sized by the occupancy query.  When a
+ *   sequence is split into more than four pieces, every cluster holding a piece waits for all the
+ *   others (the sliced merge), which needs every cluster resident at once.  The launcher uses that
+ *   merge only when the occupancy query confirmed the wave; setting MLA_DECODE_SLICED_MERGE=0 in
+ *   the environment turns it off (for GPUs shared with MPS clients or other processes' persistent
+ *   kernels).  Without it the last piece to finish merges all the others.  A wait that runs out
+ *   (SMs held by another context for longer than the limit) stores MLA_ERR_TIMEOUT in dev_err.
  */
 mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
                              const void* q_tilde, int64_t ldqt, const void* q_pe, int64_t ldqp,
@@ -155,6 +162,7 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
  *   workspace                        mla_decode_workspace_size(dims, dtype, B * T, n_max, 0) bytes
  * bf16 DeepSeek dimensions only, no top-k set for T > 1 (MLA_ERR_UNSUPPORTED).  Each token runs as
  * its own query group over the shared cache rows of its sequence.  Asynchronous on `stream`.
+ * Residency and MLA_DECODE_SLICED_MERGE as for mla_decode_absorb.
  */
 mla_status mla_decode_absorb_multi(mla_dims dims, mla_dtype dtype, int32_t B, int32_t T,
                                    const void* q_tilde, int64_t ldqt, const void* q_pe, int64_t ldqp,
