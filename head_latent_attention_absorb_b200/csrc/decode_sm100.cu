@@ -69,7 +69,8 @@ constexpr int kSoftmaxWarps = 8;                // two per TMEM lane quadrant
 constexpr int kPvWarp = 2;                      // the warp that issues the P*V MMAs
 constexpr int kAWarp0 = 3;                      // 4 exchange warps, one per TMEM lane quadrant
 constexpr int kBWarp0 = 7;                      // 8 softmax warps
-constexpr int kThreads = 32 * (kBWarp0 + kSoftmaxWarps);
+constexpr int kGatherWarp = kBWarp0 + kSoftmaxWarps;  // top-k decode: copies keys [32, 64) of each tile
+constexpr int kThreads = 32 * (kGatherWarp + 1);  // 512 threads x 128 registers: the whole register file
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 0, kColS = 256, kColP = 320, kColQ = 352;  // Q: 128 + 16 columns
 constexpr float kRescaleThreshold = 8.0f;       // log2 units
@@ -343,6 +344,32 @@ __device__ void plan_range(const Params& p, int c, Smem& sm, int lane) {
   }
 }
 
+// Top-k decode: copies keys [32 h, 32 h + 32) of a gathered tile (lane l holds the cache row of key
+// 32 h + l) with 16-byte cp.async into exactly the layout the TMA boxes would give: latent slab s,
+// key k, chunk c at s * 8 KB + 128 k + 16 (c ^ (k & 7)); rotary key k, chunk c at
+// 32 KB + 64 k + 16 (c ^ ((k >> 1) & 3)).  Eight lanes cover one 128-byte row, so every instruction
+// reads four whole rows and hits distinct banks.  Each lane's copies then count once on `bar`.
+__device__ __forceinline__ void gather_half(const Params& p, int row_of_lane, int h, uint32_t dst, uint32_t bar,
+                                            uint32_t rank, int lane) {
+#pragma unroll
+  for (int g = 0; g < 8; ++g) {
+    const int kl = 4 * g + (lane >> 3), ch = lane & 7, key = 32 * h + kl;
+    const int r = __shfl_sync(0xffffffffu, row_of_lane, kl);
+    const __nv_bfloat16* src = p.c_kv_base + (int64_t)r * p.ckv_row + 256 * rank + 8 * ch;
+    const uint32_t d = dst + key * 128 + ((ch ^ (key & 7)) << 4);
+#pragma unroll
+    for (int sl = 0; sl < 4; ++sl) cp_async_16(d + sl * kSlabBytes, src + 64 * sl);
+  }
+#pragma unroll
+  for (int g = 0; g < 4; ++g) {
+    const int kl = 8 * g + (lane >> 2), ch = lane & 3, key = 32 * h + kl;
+    const int r = __shfl_sync(0xffffffffu, row_of_lane, kl);
+    const __nv_bfloat16* src = p.k_r_base + (int64_t)r * p.kr_row + 32 * rank + 8 * ch;
+    cp_async_16(dst + kLatBytes + key * 64 + ((ch ^ ((key >> 1) & 3)) << 4), src);
+  }
+  cp_async_mbar_arrive(bar);
+}
+
 // Walks the segments (sequence, first tile, end tile) of this cluster's range.
 struct SegIter {
   int b, tb, t, hi, len0;
@@ -470,7 +497,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       // dense: the producer's arrive.expect_tx + the TMA bytes; sparse: one cp.async arrival per lane
-      mbar_init(smem_u32(&sm.full[s]), p.topk > 0 ? 32 : 1);
+      // of the two gathering warps
+      mbar_init(smem_u32(&sm.full[s]), p.topk > 0 ? 64 : 1);
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     // softmax-side arrivals are one per softmax warp, after a __syncwarp
@@ -519,7 +547,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   // the cluster barrier now and waits before its first remote operation.  The producer only touches
   // this CTA's memory, so it starts loading before it waits.
   asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
-  if (warp != 0) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+  if (warp != 0 && warp != kGatherWarp) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   const uint32_t tmem = sm.tmem_base;
 
   if (warp == 0) {
@@ -551,20 +579,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           q_issued = true;
         }
         const int seq_len_b = p.topk > 0 ? clamp_len(p.lengths[b], p.n_max) : 0;
-        // sparse: the positions of tile i + 1 are loaded while tile i is issued (two per lane), so
-        // no tile waits for its own index load
-        int pos_next[2] = {0, 0};
-        auto load_pos = [&](int i, int (&dst)[2]) {
-#pragma unroll
-          for (int hf = 0; hf < 2; ++hf) {
-            const int k = i * kTile + 32 * hf + lane;
-            dst[hf] = k < p.topk ? p.topk_idx[(int64_t)b * p.topk + k] : 0;
-          }
+        // sparse: the positions of keys [0, 32) of tile i + 1 are loaded while tile i is issued
+        // (one per lane), so no tile waits for its own index load
+        int pos_next = 0;
+        auto load_pos = [&](int i) {
+          const int k = i * kTile + lane;
+          return k < p.topk ? p.topk_idx[(int64_t)b * p.topk + k] : 0;
         };
-        if (p.topk > 0) load_pos(begin, pos_next);
+        if (p.topk > 0) pos_next = load_pos(begin);
         for (int i = begin; i < end && ok; ++i, ++it) {
-          int pos_cur[2] = {pos_next[0], pos_next[1]};
-          if (p.topk > 0 && i + 1 < end) load_pos(i + 1, pos_next);
+          const int pos_cur = pos_next;
+          if (p.topk > 0 && i + 1 < end) pos_next = load_pos(i + 1);
           const uint32_t st = it % kStages, ph = (it / kStages) & 1u;
           if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs))) {
             if (lane == 0) fail_timeout(sm, p.err);
@@ -584,40 +609,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           } else {
             // rows of the 2-D caches: b * n_max + position; positions past the top-k set (the last
             // tile's tail, zeroed before use) and invalid ones (flagged) read position 0
-            int rows[2];
-#pragma unroll
-            for (int hf = 0; hf < 2; ++hf) {
-              int pos = 0;
-              if (i * kTile + 32 * hf + lane < p.topk) {
-                pos = pos_cur[hf];
-                if (pos < 0 || pos >= seq_len_b) {
-                  raise_error(p.err, MLA_ERR_INDEX);
-                  pos = 0;
-                }
+            int pos = 0;
+            if (i * kTile + lane < p.topk) {
+              pos = pos_cur;
+              if (pos < 0 || pos >= seq_len_b) {
+                raise_error(p.err, MLA_ERR_INDEX);
+                pos = 0;
               }
-              rows[hf] = b * p.n_max + pos;
             }
-            // Each lane copies 16-byte chunks (cp.async) straight into the swizzled layout a TMA box
-            // would produce: latent slab s, key k, chunk c at s * 8 KB + 128 k + 16 (c ^ (k & 7));
-            // rotary key k, chunk c at 32 KB + 64 k + 16 (c ^ ((k >> 1) & 3)).  Eight lanes cover one
-            // 128-byte row, so every instruction reads four whole rows and hits distinct banks.
-#pragma unroll 1
-            for (int g = 0; g < kTile / 4; ++g) {
-              const int key = 4 * g + (lane >> 3), ch = lane & 7;
-              const int r0 = __shfl_sync(0xffffffffu, rows[0], key & 31), r1 = __shfl_sync(0xffffffffu, rows[1], key & 31);
-              const __nv_bfloat16* src = p.c_kv_base + (int64_t)(key < 32 ? r0 : r1) * p.ckv_row + 256 * rank + 8 * ch;
-              const uint32_t d = dst + key * 128 + ((ch ^ (key & 7)) << 4);
-#pragma unroll
-              for (int s = 0; s < 4; ++s) cp_async_16(d + s * kSlabBytes, src + 64 * s);
-            }
-#pragma unroll 1
-            for (int g = 0; g < kTile / 8; ++g) {
-              const int key = 8 * g + (lane >> 2), ch = lane & 3;
-              const int r0 = __shfl_sync(0xffffffffu, rows[0], key & 31), r1 = __shfl_sync(0xffffffffu, rows[1], key & 31);
-              const __nv_bfloat16* src = p.k_r_base + (int64_t)(key < 32 ? r0 : r1) * p.kr_row + 32 * rank + 8 * ch;
-              cp_async_16(dst + kLatBytes + key * 64 + ((ch ^ ((key >> 1) & 3)) << 4), src);
-            }
-            cp_async_mbar_arrive(bar);  // this lane's copies of the tile, counted on full[st]
+            gather_half(p, b * p.n_max + pos, 0, dst, bar, rank, lane);
           }
           __syncwarp();
         }
@@ -811,6 +811,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       wait_or_fail(smem_u32(&sm.x_free[t & 1u]), ((t >> 1) + 1u) & 1u, true);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&sm.xch_drained));
+  } else if (warp == kGatherWarp) {
+    // ------------------------------------------------------------------ second gathering warp
+    // Top-k decode only: keys [32, 64) of every tile, in step with the producer (same stage ring;
+    // the stage's full barrier counts both warps' lanes).  Like the producer it touches only this
+    // CTA's memory, so it waits on the cluster barrier at the end.
+    if (p.topk > 0) {
+      SegIter seg(sm, p);
+      int b, begin, end, len, base;
+      bool whole;
+      uint32_t it = 0;
+      bool ok = true, waited = false;
+      while (ok && seg.next(b, begin, end, len, whole, base)) {
+        if (!waited) {
+          griddep_wait();  // the top-k indices may be the preceding kernel's output
+          waited = true;
+        }
+        const int seq_len_b = clamp_len(p.lengths[b], p.n_max);
+        auto load_pos = [&](int i) {
+          const int k = i * kTile + 32 + lane;
+          return k < p.topk ? p.topk_idx[(int64_t)b * p.topk + k] : 0;
+        };
+        int pos_next = load_pos(begin);
+        for (int i = begin; i < end && ok; ++i, ++it) {
+          const int pos_cur = pos_next;
+          if (i + 1 < end) pos_next = load_pos(i + 1);
+          const uint32_t st = it % kStages, ph = (it / kStages) & 1u;
+          if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs))) {
+            if (lane == 0) fail_timeout(sm, p.err);
+            ok = false;
+            break;
+          }
+          int pos = 0;
+          if (i * kTile + 32 + lane < p.topk) {
+            pos = pos_cur;
+            if (pos < 0 || pos >= seq_len_b) {
+              raise_error(p.err, MLA_ERR_INDEX);
+              pos = 0;
+            }
+          }
+          gather_half(p, b * p.n_max + pos, 1, smem_u32(stages + st * kStageBytes), smem_u32(&sm.full[st]), rank, lane);
+          __syncwarp();
+        }
+      }
+    }
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   } else {
     // ------------------------------------------------------------------ softmax warps (kBWarp0..)
     griddep_wait();  // they read the absorbed query and write the context / workspace
@@ -830,6 +876,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto warp_arrive = [&](uint32_t bar) {
       __syncwarp();
       if (lane == 0) mbar_arrive(bar);
+    };
+    // Staged stores, for the range's last segment (no cache tile lands in the stage buffers any more):
+    // this warp's 32 heads x 16 chunks of 16 bytes go through shared memory (its 8 KB at
+    // stages + 72 KB, past a bulk-loaded partial and its (m, l) pairs; chunk c of lane l's head at
+    // l * 256 + 16 (c ^ (l & 15)), conflict-free both ways), then every store instruction writes two
+    // whole 256-byte head rows instead of 32 scattered 16-byte pieces.
+    const uint32_t stg_out = smem_u32(stages) + 73728u + (uint32_t)sw * 8192u;
+    auto stage_chunk = [&](int c, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+      st_shared_v4_b32(stg_out + lane * 256 + ((c ^ (lane & 15)) << 4), x, y, z, w);
+    };
+    // dst(hl, cc): global address of chunk cc (of 16) of local head hl (head quad * 32 + hl)
+    auto flush_staged = [&](auto dst) {
+      __syncwarp();
+#pragma unroll 4
+      for (int i = 0; i < 16; ++i) {
+        const int hl = 2 * i + (lane >> 4), cc = lane & 15;
+        *dst(hl, cc) = ld_shared_v4_b32(stg_out + hl * 256 + ((cc ^ (hl & 15)) << 4));
+      }
+      __syncwarp();
     };
     SegIter seg(sm, p);
     int b, begin, end, len, base;
@@ -1012,6 +1077,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       warp_arrive(smem_u32(&sm.sum_bar));
       if (!wait_or_fail(smem_u32(&sm.sum_bar), nseg & 1u, false)) break;
       const float l_tot = l_run + sm.lsum[half ^ 1][h];
+      const bool staged = (base + end >= sm.hi);  // the range's last segment: stage buffers idle
+      // ctx chunk cc of local head hl, this CTA's latent half and this warp's 128 features
+      auto ctx_chunk = [&](int hl, int cc) {
+        return reinterpret_cast<uint4*>(p.ctx + ((int64_t)b * kNH + quad * 32 + hl) * kDC + 256 * rank + 128 * half) + cc;
+      };
       if (whole) {
         const float inv = 1.f / l_tot;
         __nv_bfloat16* out = p.ctx + ((int64_t)b * kNH + h) * kDC + 256 * rank + 128 * half;
@@ -1026,8 +1096,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             w[k] = pack_bf16x2(__uint_as_float(r[2 * k]) * inv, __uint_as_float(r[2 * k + 1]) * inv);
           uint4* dst = reinterpret_cast<uint4*>(out + c * 32);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          for (int v = 0; v < 4; ++v) {
+            if (staged) stage_chunk(4 * c + v, w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+            else dst[v] = make_uint4(w[4 * v], w[4 * v + 1], w[4 * v + 2], w[4 * v + 3]);
+          }
         }
+        if (staged) flush_staged(ctx_chunk);
         if (rank == 0 && half == 0 && p.lse != nullptr)
           p.lse[(int64_t)b * kNH + h] = (m_run + log2f(l_tot)) * 0.69314718055994531f;
       } else {
@@ -1063,13 +1137,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int v = 0; v < 4; ++v) {
               const int chunk = 16 * half + 4 * c + v;
-              row[chunk ^ cswz] = make_uint4(
-                  pack_bf16x2(__uint_as_float(r[8 * v]) * inv_own, __uint_as_float(r[8 * v + 1]) * inv_own),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_own, __uint_as_float(r[8 * v + 3]) * inv_own),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_own, __uint_as_float(r[8 * v + 5]) * inv_own),
-                  pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_own, __uint_as_float(r[8 * v + 7]) * inv_own));
+              const uint32_t x = pack_bf16x2(__uint_as_float(r[8 * v]) * inv_own, __uint_as_float(r[8 * v + 1]) * inv_own);
+              const uint32_t y = pack_bf16x2(__uint_as_float(r[8 * v + 2]) * inv_own, __uint_as_float(r[8 * v + 3]) * inv_own);
+              const uint32_t z = pack_bf16x2(__uint_as_float(r[8 * v + 4]) * inv_own, __uint_as_float(r[8 * v + 5]) * inv_own);
+              const uint32_t w = pack_bf16x2(__uint_as_float(r[8 * v + 6]) * inv_own, __uint_as_float(r[8 * v + 7]) * inv_own);
+              if (staged) stage_chunk(4 * c + v, x, y, z, w);
+              else row[chunk ^ cswz] = make_uint4(x, y, z, w);
             }
           }
+          if (staged)
+            flush_staged([&](int hl, int cc) {
+              const int hh = quad * 32 + hl;
+              return reinterpret_cast<uint4*>(p.ws_o) + (((int64_t)own * 2 + rank) * kNH + hh) * 32 +
+                     ((16 * half + cc) ^ (hh & 15));
+            });
           if (half == 0) p.ws_ml[((int64_t)own * 2 + rank) * kNH + h] = make_float2(m_run, l_tot);
           __threadfence();
           warp_arrive(smem_u32(&sm.pub_bar));
@@ -1485,10 +1566,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             }
             uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              d4[v] = make_uint4(pack_bf16x2(acc[8 * v], acc[8 * v + 1]), pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]),
-                                 pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]));
+            for (int v = 0; v < 4; ++v) {
+              const uint32_t x = pack_bf16x2(acc[8 * v], acc[8 * v + 1]), y = pack_bf16x2(acc[8 * v + 2], acc[8 * v + 3]);
+              const uint32_t z = pack_bf16x2(acc[8 * v + 4], acc[8 * v + 5]), w = pack_bf16x2(acc[8 * v + 6], acc[8 * v + 7]);
+              if (bulk) stage_chunk(4 * c + v, x, y, z, w);  // (bulk: the range's last segment)
+              else d4[v] = make_uint4(x, y, z, w);
+            }
           }
+          if (bulk) flush_staged(ctx_chunk);
           if (rank == 0 && half == 0 && p.lse != nullptr)
             p.lse[(int64_t)b * kNH + h] = (M + log2f(L)) * 0.69314718055994531f;
           // the flags go back to zero for the next launch (which may reuse this launch's epoch when
