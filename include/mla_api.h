@@ -131,7 +131,7 @@ int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32
  *   dev_err  NULL or a device int32 flag; MLA_ERR_LENGTH / MLA_ERR_INDEX are stored there
  * Asynchronous on `stream`.
  * Residency: the kernel is one persistent wave of CTA pairs sized by the occupancy query.  When a
- *   sequence is split into more than four pieces, every cluster holding a piece waits for all the
+ *   sequence is split into more than two pieces, every cluster holding a piece waits for all the
  *   others (the sliced merge), which needs every cluster resident at once.  The launcher uses that
  *   merge only when the occupancy query confirmed the wave; setting MLA_DECODE_SLICED_MERGE=0 in
  *   the environment turns it off (for GPUs shared with MPS clients or other processes' persistent

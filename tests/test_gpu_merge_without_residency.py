@@ -13,7 +13,7 @@ import torch
 
 import oracle as O
 from head_latent_attention_absorb_b200 import api
-from head_latent_attention_absorb_b200.configs import RAGGED_LONG, V3_DECODE
+from head_latent_attention_absorb_b200.configs import RAGGED_LONG, SPARSE_V32, V3_DECODE
 from head_latent_attention_absorb_b200.inputs import make_decode_inputs
 
 from _util import check_close
@@ -98,3 +98,32 @@ def test_multi_token_decode_long_sequence(dev, monkeypatch):
         for name, ctx, lse in (("sliced", ctx_s, lse_s), ("last-arrival", ctx_l, lse_l)):
             check_close(ctx[0, s], want_ctx, torch.bfloat16, f"{name} merge token {s} ctx")
             check_close(lse[s], want_lse, torch.bfloat16, f"{name} merge token {s} lse")
+
+
+def test_topk_decode_four_partials(dev, monkeypatch):
+    """Top-k decode, B = 16 sequences of 2048 selected rows over 74 clusters: four partials per
+    sequence.  Sliced (every cluster merges a quarter of the heads) and, with the sliced merge off,
+    the last cluster bulk-loading the three others; both against the oracle on two sequences."""
+    cfg = SPARSE_V32
+    x = make_decode_inputs(cfg)
+    qt = torch.from_numpy(O.absorb_q(x["q_nope"], x["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v)).to(torch.bfloat16)
+    cache = x["cache"].to(dev)
+    topk = x["topk"].to(dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def call():
+        lse = torch.empty((cfg.B, cfg.n_h), dtype=torch.float32, device=dev)
+        ctx = api.mla_decode_absorb(cfg.dims, qt.to(dev), x["q_pe"].to(dev), cache[..., :cfg.d_c],
+                                    cache[..., cfg.d_c:], x["lengths"].to(dev), cfg.scale, topk_idx=topk,
+                                    lse=lse, dev_err=err)
+        return ctx.clone(), lse.clone()
+
+    (ctx_s, lse_s), (ctx_l, lse_l) = _both_merges(monkeypatch, call)
+    assert api.mla_get_device_error(err) == 0
+    for b in (0, cfg.B - 1):
+        L = int(x["lengths"][b])
+        want_ctx, want_lse, _ = O.latent_attention(qt[b], x["q_pe"][b], x["c_kv"][b, :L], x["k_r"][b, :L],
+                                                   cfg.scale, x["topk"][b].numpy())
+        for name, ctx, lse in (("sliced", ctx_s, lse_s), ("last-arrival", ctx_l, lse_l)):
+            check_close(ctx[b], want_ctx, torch.bfloat16, f"{name} merge ctx b={b}")
+            check_close(lse[b], want_lse, torch.bfloat16, f"{name} merge lse b={b}")
