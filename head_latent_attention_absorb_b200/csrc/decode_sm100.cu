@@ -561,7 +561,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       SegIter seg(sm, p);
       int b, begin, end, len, base;
       bool whole;
-      uint32_t it = 0;
+      uint32_t it = 0, nseg_p = 0;
       bool ok = true, q_issued = false;
       while (ok && seg.next(b, begin, end, len, whole, base)) {
         if (!q_issued) {
@@ -620,7 +620,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             gather_half(p, b * p.n_max + pos, 0, dst, bar, rank, lane);
           }
           __syncwarp();
+          if (i == end - 1 && !whole) {
+            // The segment's last tile is on its way: count this cluster's arrival for the sequence
+            // (per latent half) now.  An atomic takes about a microsecond while HBM is busy; here it
+            // overlaps the last tiles' work instead of delaying the epilogue.  The epilogue reads the
+            // decision (and the slot list) after waiting on last_bar.  A later segment's decision
+            // waits until that segment's query is in (q_full), i.e. until the previous segment's
+            // epilogue is done with the slot list.
+            int okq = 1;
+            if (lane == 0) {
+              if (nseg_p > 0 && !mbar_wait(smem_u32(&sm.q_full), nseg_p & 1u, abort_flag, kWaitLimitNs)) okq = 0;
+              if (okq) {
+                const int ns = list_slots(p, sm, base, tiles_of(len));
+                // up to p.slice_above partials (kMergeLastMax = 2 when the whole grid is resident,
+                // else any number) the last cluster to arrive merges them all; with more, every
+                // cluster publishes and then merges its own slice of the heads (with three or four
+                // partials the slices run in parallel: top-k call 43.8 -> 41.0 us against one
+                // merging cluster)
+                sm.is_last = ns > p.slice_above ? 0 : (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0);
+                mbar_arrive(smem_u32(&sm.last_bar));
+              } else {
+                fail_timeout(sm, p.err);
+              }
+            }
+            if (!__shfl_sync(0xffffffffu, okq, 0)) {
+              ok = false;
+              break;
+            }
+          }
         }
+        ++nseg_p;
       }
       // drain: every load issued must have landed before the CTA may exit
       if (lane == 0) {
@@ -1107,19 +1136,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       } else {
         // ---- partial: the last of the sequence's clusters to arrive (per latent half) merges every
         // partial into ctx; the others publish (O, m, l) in their segment's slot and then raise the
-        // slot's ready flag.  Counting the arrival first means the merger never writes its own
-        // partial, and every cluster it then waits for has already arrived (so it is running) and
-        // needs nothing from the merger, so the wait ends.
+        // slot's ready flag.  Counting the arrival first (the producer does, at the segment's last
+        // tile) means the merger never writes its own partial, and every cluster it then waits for
+        // has already arrived (so it is running) and needs nothing from the merger, so the wait
+        // ends.
         const int own = 2 * cl + (first_seg ? 0 : 1);
-        if (sw == 0 && lane == 0) {
-          const int ns = list_slots(p, sm, base, tiles_of(len));
-          // up to p.slice_above partials (kMergeLastMax = 2 when the whole grid is resident, else
-          // any number) the last cluster to arrive merges them all; with more, every cluster
-          // publishes and then merges its own slice of the heads (with three or four partials the
-          // slices run in parallel: top-k call 43.8 -> 41.0 us against one merging cluster)
-          sm.is_last = ns > p.slice_above ? 0 : (arrive_last(p.ws_ctr + 2 * (int64_t)b + rank, p.epoch, ns, p.err) ? 1 : 0);
-          mbar_arrive(smem_u32(&sm.last_bar));
-        }
+        // the producer counted the arrival when it issued the segment's last tile
         if (!wait_or_fail(smem_u32(&sm.last_bar), npart & 1u, false)) break;
         ++npart;
         // A partial is this segment's context normalised by its own softmax sum, in bf16: head-major
