@@ -37,7 +37,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch on this workload,
 # from one ncu capture of the decode kernel, valid only for the kernel source it was taken on
 # (sha256 prefix of csrc/decode_sm100.cu).
-DECODE_TRAFFIC = {"bytes": 155_830_528 + 3_131_904, "source_sha256": "67d9510d3f1a9f81"}
+DECODE_TRAFFIC = {"bytes": 155_841_536 + 3_184_128, "source_sha256": "a94e21789ec2ca7d"}
 
 
 def decode_traffic():
