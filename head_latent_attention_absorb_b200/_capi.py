@@ -39,6 +39,9 @@ SIGNATURES = {
                                   c_vp, c_i64, c_i64, c_vp, c_i64, c_i64,
                                   c_i32, c_vp, c_vp, c_i32,
                                   c_f32, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "mla_decode_absorb_fp8kv": (c_i32, [MLADims, c_i32, c_vp, c_i64, c_vp, c_i64,
+                                        c_vp, c_i64, c_i64, c_vp, c_i64, c_i64, c_vp, c_i64, c_i64,
+                                        c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "mla_decode_absorb_multi": (c_i32, [MLADims, c_i32, c_i32, c_i32,
                                         c_vp, c_i64, c_vp, c_i64,
                                         c_vp, c_i64, c_i64, c_vp, c_i64, c_i64,

@@ -111,6 +111,37 @@ def mla_decode_absorb(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_kv: tor
     return ctx
 
 
+def mla_decode_absorb_fp8kv(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c8: torch.Tensor,
+                            kv_scale: torch.Tensor, k_r: torch.Tensor, lengths: torch.Tensor, scale: float,
+                            ctx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                            workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                            stream=None) -> torch.Tensor:
+    """The absorbed decode over an FP8 latent cache: c8 [B, n_max, d_c] uint8 E4M3 codes, kv_scale
+    [B, n_max, d_c / 128] float32 (one scale per 128 latent features of a row), k_r [B, n_max, d_r]
+    bf16; all three may be strided views (e.g. of one packed 656-byte row)."""
+    d = _dims(dims)
+    B, n_max = c8.shape[0], c8.shape[1]
+    ldqt, ldqp = _headrows(q_tilde, "q_tilde"), _headrows(q_pe, "q_pe")
+    for t, n in ((c8, "c8"), (kv_scale, "kv_scale"), (k_r, "k_r")):
+        _rows(t, n)
+    if c8.dtype != torch.uint8 or kv_scale.dtype != torch.float32:
+        raise TypeError("c8 must be uint8 and kv_scale float32")
+    if lengths.dtype != torch.int32:
+        raise TypeError("lengths must be int32")
+    if ctx is None:
+        ctx = torch.empty((B, d.n_h, d.d_c), dtype=q_tilde.dtype, device=q_tilde.device)
+    if workspace is None:
+        nbytes = mla_decode_workspace_size(d, q_tilde.dtype, B, n_max, 0)
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=q_tilde.device)
+    check(lib().mla_decode_absorb_fp8kv(
+        d, B, _ptr(q_tilde), ldqt, _ptr(q_pe), ldqp,
+        _ptr(c8), c8.stride(0), c8.stride(1), _ptr(kv_scale), kv_scale.stride(0), kv_scale.stride(1),
+        _ptr(k_r), k_r.stride(0), k_r.stride(1), n_max, _ptr(lengths), float(scale),
+        _ptr(ctx), _ptr(lse), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _ptr(dev_err), _stream(stream)), "mla_decode_absorb_fp8kv")
+    return ctx
+
+
 def mla_decode_absorb_multi(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_kv: torch.Tensor,
                             k_r: torch.Tensor, lengths: torch.Tensor, scale: float,
                             ctx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,

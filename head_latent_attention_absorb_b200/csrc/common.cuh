@@ -63,6 +63,10 @@ struct DecodeArgs {
   void* ctx;
   float* lse;
   int32_t* err;
+  // FP8 latent cache (mla_decode_absorb_fp8kv): e4m3 rows replace c_kv; strides in bytes for c8 and
+  // in floats for kv_scale (one fp32 scale per 128 latent features of a row)
+  const void* c8 = nullptr;        int64_t c8_b = 0, c8_r = 0;
+  const float* kv_scale = nullptr; int64_t sc_b = 0, sc_r = 0;
 };
 
 struct PrefillArgs {

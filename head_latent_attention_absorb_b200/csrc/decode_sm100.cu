@@ -32,6 +32,7 @@
 //   MLA_ERR_TIMEOUT, drains and returns.
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <math.h>
 #include <string.h>
 
@@ -63,6 +64,14 @@ static_assert(kQLatBytes == 4 * kXBytes, "the first query is staged in the four 
 constexpr int kXOff = kStages * kStageBytes;    // shared-memory layout: stages | exchange | q rope | Smem
 constexpr int kQRopeOff = kXOff + 4 * kXBytes;
 constexpr int kSmemOff = kQRopeOff + kQRopeBytes;
+// FP8 latent cache: three bf16 stages, and behind them two raw slots of one tile's e4m3 latent half
+// (64 rows x 256 bytes) plus its scales (64 rows x 4 fp32), which the conversion warp turns into the
+// stage's bf16 tile
+constexpr int kStagesFp8 = 3;
+constexpr int kRawOff = kStagesFp8 * kStageBytes;
+constexpr int kRawLatBytes = kTile * 256;
+constexpr int kRawSlotBytes = kRawLatBytes + kTile * 16;
+static_assert(kRawOff + 2 * kRawSlotBytes <= kXOff, "FP8 raw slots overlap the exchange buffers");
 constexpr int kMaxClusters = 160;               // partial-slot list capacity (2 slots per cluster)
 constexpr int kMergeLastMax = 2;                // up to this many partials the last cluster merges alone
 constexpr int kSoftmaxWarps = 8;                // two per TMEM lane quadrant
@@ -103,6 +112,9 @@ struct Params {
   unsigned long long* ws_ready;  // [2 n_clusters slots][2 halves] partial published: the writer's epoch
   unsigned long long epoch;    // unique per launch, never 0, < 2^56
   int32_t* err;
+  // FP8 latent cache (the kFp8 kernel): e4m3 latent rows and their per-128-feature fp32 scales
+  CUtensorMap tm_c8;   // 3-D (512 bytes, n_max, B), box (256, 64, 1), no swizzle
+  CUtensorMap tm_sc;   // 3-D (4 scales, n_max, B), box (4, 64, 1)
 };
 
 struct Smem {
@@ -116,6 +128,7 @@ struct Smem {
   uint64_t mrg_full2[2], mrg_empty2[2];  // streamed merge of several partials (double-buffered)
   uint64_t xch_drained;            // the peer has read every partial score this CTA sent
   uint64_t mrg_done;               // every softmax warp finished its share of a sliced merge
+  uint64_t raw_full[2], raw_empty[2];  // FP8 cache: raw tile landed / converted
   float red[2][2][kNH];            // [tile parity][key half][head] partial row max
   float lsum[2][kNH];              // [key half][head] partial softmax sum
   int16_t slots[kMaxClusters];     // partial slots of the sequence being merged
@@ -476,8 +489,11 @@ __device__ bool wait_flag(const unsigned long long* f, unsigned long long want, 
   }
 }
 
+template <bool kFp8>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ Params p) {
+  // stages of the ring: four bf16 tiles, or three for the FP8 cache (its raw slots take the fourth)
+  constexpr int kNS = kFp8 ? kStagesFp8 : kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stages = smem;
@@ -498,7 +514,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       // dense: the producer's arrive.expect_tx + the TMA bytes; sparse: one cp.async arrival per lane
       // of the two gathering warps
-      mbar_init(smem_u32(&sm.full[s]), p.topk > 0 ? 64 : 1);
+      // FP8 cache: the producer's arrive.expect_tx for the rotary slab + the conversion warp's arrival
+      mbar_init(smem_u32(&sm.full[s]), kFp8 ? 2 : (p.topk > 0 ? 64 : 1));
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     // softmax-side arrivals are one per softmax warp, after a __syncwarp
@@ -527,6 +544,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(smem_u32(&sm.mrg_full2[i]), 1);
       mbar_init(smem_u32(&sm.mrg_empty2[i]), kSoftmaxWarps);
+      mbar_init(smem_u32(&sm.raw_full[i]), 1);
+      mbar_init(smem_u32(&sm.raw_empty[i]), 1);
     }
     sm.abort = 0;
     fence_mbar_init();
@@ -534,6 +553,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     prefetch_tensormap(&p.tm_kr);
     prefetch_tensormap(&p.tm_q);
     prefetch_tensormap(&p.tm_qp);
+    if (kFp8) {
+      prefetch_tensormap(&p.tm_c8);
+      prefetch_tensormap(&p.tm_sc);
+    }
   }
   if (warp == 0) plan_range(p, cl, sm, lane);
   if (warp == 1) {
@@ -590,7 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = begin; i < end && ok; ++i, ++it) {
           const int pos_cur = pos_next;
           if (p.topk > 0 && i + 1 < end) pos_next = load_pos(i + 1);
-          const uint32_t st = it % kStages, ph = (it / kStages) & 1u;
+          const uint32_t st = it % kNS, ph = (it / kNS) & 1u;
           if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs))) {
             if (lane == 0) fail_timeout(sm, p.err);
             ok = false;
@@ -598,7 +621,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           const uint32_t dst = smem_u32(stages + st * kStageBytes);
           const uint32_t bar = smem_u32(&sm.full[st]);
-          if (p.topk == 0) {
+          if (kFp8) {
+            // the rotary half straight into the stage; the e4m3 latent half and its scales into raw
+            // slot it & 1 once the conversion warp has read that slot's previous tile
+            int okr = 1;
+            if (lane == 0) {
+              mbar_arrive_expect_tx(bar, kRopeBytes);
+              tma_load_3d(dst + kLatBytes, &p.tm_kr, bar, 32 * (int)rank, i * kTile, b, pol);
+              const uint32_t rs = it & 1u, rb = smem_u32(&sm.raw_full[rs]);
+              if (mbar_wait(smem_u32(&sm.raw_empty[rs]), ((it >> 1) & 1u) ^ 1u, abort_flag, kWaitLimitNs)) {
+                const uint32_t raw = smem_u32(smem + kRawOff + rs * kRawSlotBytes);
+                mbar_arrive_expect_tx(rb, kRawSlotBytes);
+                tma_load_3d(raw, &p.tm_c8, rb, 256 * (int)rank, i * kTile, b, pol);
+                tma_load_3d(raw + kRawLatBytes, &p.tm_sc, rb, 0, i * kTile, b, pol);
+              } else {
+                fail_timeout(sm, p.err);
+                okr = 0;
+              }
+            }
+            if (!__shfl_sync(0xffffffffu, okr, 0)) {
+              ok = false;
+              break;
+            }
+          } else if (p.topk == 0) {
             if (lane == 0) {
               mbar_arrive_expect_tx(bar, kStageBytes);
 #pragma unroll
@@ -653,9 +698,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       // drain: every load issued must have landed before the CTA may exit
       if (lane == 0) {
-        const uint32_t first = it > (uint32_t)kStages ? it - kStages : 0;
+        const uint32_t first = it > (uint32_t)kNS ? it - kNS : 0;
         for (uint32_t k = first; k < it; ++k)
-          mbar_wait(smem_u32(&sm.full[k % kStages]), (k / kStages) & 1u, abort_flag, kWaitLimitNs);
+          mbar_wait(smem_u32(&sm.full[k % kNS]), (k / kNS) & 1u, abort_flag, kWaitLimitNs);
         if (q_issued) mbar_wait(smem_u32(&sm.q_tma), 0, abort_flag, kWaitLimitNs);
       }
     }
@@ -701,9 +746,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     };
     // S(t) = Q K(t)^T over this CTA's 288 features
     auto issue_qk = [&](uint32_t t, int tile_in_seq) {
-      const uint32_t st = t % kStages;
-      if (!wait_or_fail(smem_u32(&sm.full[st]), (t / kStages) & 1u, false)) return;
-      if (p.topk > 0) fence_proxy_async_smem();  // rows copied by cp.async (generic proxy)
+      const uint32_t st = t % kNS;
+      if (!wait_or_fail(smem_u32(&sm.full[st]), (t / kNS) & 1u, false)) return;
+      if (p.topk > 0 || kFp8) fence_proxy_async_smem();  // rows written through the generic proxy
       const int valid = len - tile_in_seq * kTile;
       if (valid < kTile) {  // rows past the sequence end: zero them so 0 * garbage cannot occur
         uint8_t* sbase = stages + st * kStageBytes;
@@ -739,8 +784,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     auto issue_pv = [&](uint32_t t, bool first_of_seg) {
       if (!wait_or_fail(smem_u32(&sm.p_full), t & 1u, false)) return;
       tc_fence_after();
-      if (p.topk > 0) fence_proxy_async_smem();
-      const uint32_t st = t % kStages;
+      if (p.topk > 0 || kFp8) fence_proxy_async_smem();
+      const uint32_t st = t % kNS;
       if (lane == 0) {
         const uint32_t base = smem_u32(stages + st * kStageBytes);
 #pragma unroll
@@ -840,6 +885,57 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       wait_or_fail(smem_u32(&sm.x_free[t & 1u]), ((t >> 1) + 1u) & 1u, true);
     __syncwarp();
     if (lane == 0) mbar_arrive(smem_u32(&sm.xch_drained));
+  } else if (kFp8 && warp == kGatherWarp) {
+    // ------------------------------------------------------------------ FP8 cache: conversion warp
+    // Every tile: wait for its raw slot (e4m3 latent half + scales) and for its stage, write the
+    // dequantised latent as bf16 into the stage in exactly the layout the TMA boxes of the bf16
+    // cache give (slab s, row r, 16-byte chunk c at s * 8 KB + 128 r + 16 (c ^ (r & 7))), then release
+    // both.  Value = e4m3 code * the row's fp32 scale of its 128-feature block, rounded to bf16.
+    // Lane l converts chunk l (features 8 l .. 8 l + 7 of this CTA's half) of every row.
+    SegIter seg(sm, p);
+    int b, begin, end, len, base;
+    bool whole;
+    uint32_t it = 0;
+    bool ok = true;
+    const int blk = 2 * (int)rank + (lane >> 4);
+    const uint32_t out_off = (uint32_t)(lane >> 3) * kSlabBytes, chunk = (uint32_t)(lane & 7);
+    while (ok && seg.next(b, begin, end, len, whole, base)) {
+      for (int i = begin; i < end && ok; ++i, ++it) {
+        const uint32_t st = it % kNS, rs = it & 1u;
+        const bool got = mbar_wait(smem_u32(&sm.raw_full[rs]), (it >> 1) & 1u, abort_flag, kWaitLimitNs) &&
+                         mbar_wait(smem_u32(&sm.empty[st]), ((it / kNS) & 1u) ^ 1u, abort_flag, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) fail_timeout(sm, p.err);
+          ok = false;
+          break;
+        }
+        const uint8_t* raw = smem + kRawOff + rs * kRawSlotBytes;
+        const uint32_t dst = smem_u32(stages + st * kStageBytes) + out_off;
+#pragma unroll 4
+        for (int r = 0; r < kTile; ++r) {
+          const uint2 w = *reinterpret_cast<const uint2*>(raw + r * 256 + lane * 8);
+          const float sc = reinterpret_cast<const float*>(raw + kRawLatBytes + r * 16)[blk];
+          uint32_t o[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t word = j < 2 ? w.x : w.y;
+            const __half2_raw hr =
+                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((word >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            o[j] = pack_bf16x2(f.x * sc, f.y * sc);
+          }
+          st_shared_v4_b32(dst + r * 128 + ((chunk ^ (uint32_t)(r & 7)) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&sm.full[st]));
+          mbar_arrive(smem_u32(&sm.raw_empty[rs]));
+        }
+      }
+    }
+    __syncwarp();
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
   } else if (warp == kGatherWarp) {
     // ------------------------------------------------------------------ second gathering warp
     // Top-k decode only: keys [32, 64) of every tile, in step with the producer (same stage ring;
@@ -865,7 +961,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         for (int i = begin; i < end && ok; ++i, ++it) {
           const int pos_cur = pos_next;
           if (i + 1 < end) pos_next = load_pos(i + 1);
-          const uint32_t st = it % kStages, ph = (it / kStages) & 1u;
+          const uint32_t st = it % kNS, ph = (it / kNS) & 1u;
           if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.empty[st]), ph ^ 1u, abort_flag, kWaitLimitNs))) {
             if (lane == 0) fail_timeout(sm, p.err);
             ok = false;
@@ -1676,14 +1772,14 @@ Wave grid_wave() {
   if (dev >= 0 && dev < 64 && cache[dev].clusters > 0) return cache[dev];
   const int upper = max_clusters();
   Wave w{upper, false};
-  if (cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes()) ==
+  if (cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes()) ==
       cudaSuccess) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * upper);
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = smem_bytes();
     int active = 0;
-    if (cudaOccupancyMaxActiveClusters(&active, decode_kernel, &cfg) == cudaSuccess && active > 0) {
+    if (cudaOccupancyMaxActiveClusters(&active, decode_kernel<false>, &cfg) == cudaSuccess && active > 0) {
       w.clusters = active < upper ? active : upper;
       w.one_wave = true;
     }
@@ -1705,8 +1801,9 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   memset(&p, 0, sizeof(p));
   const uint64_t bstride_c = a.B > 1 ? (uint64_t)a.ckv_b * 2 : (uint64_t)a.n_max * a.ckv_r * 2;
   const uint64_t bstride_r = a.B > 1 ? (uint64_t)a.kr_b * 2 : (uint64_t)a.n_max * a.kr_r * 2;
-  if (!make_map_3d(&p.tm_ckv, a.c_kv, kDC, a.n_max, a.B, (uint64_t)a.ckv_r * 2, bstride_c, 64, kTile,
-                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+  // (the FP8 cache has no bf16 latent rows: its map is made below)
+  if ((a.c8 == nullptr && !make_map_3d(&p.tm_ckv, a.c_kv, kDC, a.n_max, a.B, (uint64_t)a.ckv_r * 2, bstride_c, 64,
+                                       kTile, CU_TENSOR_MAP_SWIZZLE_128B)) ||
       !make_map_3d(&p.tm_kr, a.k_r, kDR, a.n_max, a.B, (uint64_t)a.kr_r * 2, bstride_r, 32, kTile,
                    CU_TENSOR_MAP_SWIZZLE_64B))
     return cudaErrorInvalidValue;
@@ -1752,9 +1849,24 @@ cudaError_t decode_tc_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   p.err = a.err;
 
   const size_t smem = smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (a.c8 != nullptr) {
+    // FP8 latent cache: e4m3 rows (byte strides) and fp32 scales (4 per row), one tile's rows per box
+    const uint64_t cb = a.B > 1 ? (uint64_t)a.c8_b : (uint64_t)a.n_max * a.c8_r;
+    const uint64_t sb = a.B > 1 ? (uint64_t)a.sc_b * 4 : (uint64_t)a.n_max * a.sc_r * 4;
+    const uint64_t d8[3] = {(uint64_t)kDC, (uint64_t)a.n_max, (uint64_t)a.B}, s8[2] = {(uint64_t)a.c8_r, cb};
+    const uint64_t ds[3] = {4, (uint64_t)a.n_max, (uint64_t)a.B}, ss[2] = {(uint64_t)a.sc_r * 4, sb};
+    const uint32_t b8[3] = {256, kTile, 1}, bs[3] = {4, kTile, 1};
+    if (!make_tensor_map(&p.tm_c8, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.c8, 3, d8, s8, b8, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tensor_map(&p.tm_sc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a.kv_scale, 3, ds, ss, bs,
+                         CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_kernel<true>, dim3(2 * nc), dim3(kThreads), smem, st, p);
+  }
+  cudaError_t e = cudaFuncSetAttribute(decode_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_kernel, dim3(2 * nc), dim3(kThreads), smem, st, p);
+  return launch_pdl(decode_kernel<false>, dim3(2 * nc), dim3(kThreads), smem, st, p);
 }
 
 // ------------------------------------------------------------------------------------------

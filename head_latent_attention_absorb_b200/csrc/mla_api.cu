@@ -183,6 +183,55 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B, const vo
   return cuda_status(e, "mla_decode_absorb launch");
 }
 
+mla_status mla_decode_absorb_fp8kv(mla_dims dims, int32_t B, const void* q_tilde, int64_t ldqt, const void* q_pe,
+                                   int64_t ldqp, const void* c8, int64_t c8_bstride, int64_t c8_rstride,
+                                   const float* kv_scale, int64_t sc_bstride, int64_t sc_rstride, const void* k_r,
+                                   int64_t kr_bstride, int64_t kr_rstride, int32_t n_max, const int32_t* lengths,
+                                   float scale, void* ctx_out, float* lse_out, void* workspace, size_t ws_bytes,
+                                   int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  const mla_dtype dtype = MLA_BF16;
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0 || n_max <= 0) return fail(MLA_ERR_INVALID_ARG, "B and n_max must be positive");
+  if (!q_tilde || !q_pe || !c8 || !kv_scale || !k_r || !lengths || !ctx_out)
+    return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (ldqt < dims.d_c || ldqp < dims.d_r) return fail(MLA_ERR_INVALID_ARG, "query row stride too small");
+  if (c8_rstride < dims.d_c || kr_rstride < dims.d_r || sc_rstride < dims.d_c / 128 || c8_bstride < 0 ||
+      sc_bstride < 0 || kr_bstride < 0)
+    return fail(MLA_ERR_INVALID_ARG, "cache stride too small");
+  if ((c8_rstride % 16) || (c8_bstride % 16) || (sc_rstride % 4) || (sc_bstride % 4))
+    return fail(MLA_ERR_INVALID_ARG, "c8 strides must be multiples of 16 bytes, kv_scale strides of 4 floats");
+  if (!(scale > 0.f) || scale != scale) return fail(MLA_ERR_INVALID_ARG, "scale must be positive");
+  MLA_TRY(check_bf16_ptr(dtype, q_tilde, "q_tilde"));
+  MLA_TRY(check_bf16_ptr(dtype, q_pe, "q_pe"));
+  MLA_TRY(check_bf16_ptr(dtype, c8, "c8"));
+  MLA_TRY(check_bf16_ptr(dtype, kv_scale, "kv_scale"));
+  MLA_TRY(check_bf16_ptr(dtype, k_r, "k_r"));
+  MLA_TRY(check_bf16_ptr(dtype, ctx_out, "ctx_out"));
+  MLA_TRY(check_bf16_stride(dtype, ldqt, "ldqt"));
+  MLA_TRY(check_bf16_stride(dtype, ldqp, "ldqp"));
+  MLA_TRY(check_bf16_stride(dtype, kr_bstride, "kr_bstride"));
+  MLA_TRY(check_bf16_stride(dtype, kr_rstride, "kr_rstride"));
+  if ((int64_t)B * ((n_max + 63) / 64) >= ((int64_t)1 << 31))
+    return fail(MLA_ERR_UNSUPPORTED, "B * ceil(n_max / 64) must stay below 2^31");
+  const size_t need = mla_decode_workspace_size(dims, dtype, B, n_max, 0);
+  if (!workspace || ws_bytes < need)
+    return fail(MLA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace ? ws_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  mla::DecodeArgs a;
+  a.n_h = dims.n_h; a.d_c = dims.d_c; a.d_r = dims.d_r; a.B = B; a.n_max = n_max;
+  a.topk = 0;
+  a.q_tilde = q_tilde; a.ldqt = ldqt; a.q_pe = q_pe; a.ldqp = ldqp;
+  a.c_kv = c8; a.ckv_b = 0; a.ckv_r = 0;
+  a.k_r = k_r; a.kr_b = kr_bstride; a.kr_r = kr_rstride;
+  a.lengths = lengths; a.topk_idx = nullptr; a.scale = scale;
+  a.ctx = ctx_out; a.lse = lse_out; a.err = dev_err;
+  a.c8 = c8; a.c8_b = c8_bstride; a.c8_r = c8_rstride;
+  a.kv_scale = kv_scale; a.sc_b = sc_bstride; a.sc_r = sc_rstride;
+  return cuda_status(mla::decode_tc_launch(a, workspace, static_cast<cudaStream_t>(stream)),
+                     "mla_decode_absorb_fp8kv launch");
+}
+
 mla_status mla_decode_absorb_multi(mla_dims dims, mla_dtype dtype, int32_t B, int32_t T, const void* q_tilde,
                                    int64_t ldqt, const void* q_pe, int64_t ldqp, const void* c_kv,
                                    int64_t ckv_bstride, int64_t ckv_rstride, const void* k_r, int64_t kr_bstride,

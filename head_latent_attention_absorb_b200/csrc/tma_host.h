@@ -24,10 +24,12 @@ inline EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
-// bf16 tiled map of `rank` dimensions (innermost first); strides are in bytes for dims 1..rank-1.
-// Out-of-range elements of a box read as zero.  Returns false when the driver rejects the map.
-inline bool make_tensor_map_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                                 const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
+// Tiled map of `rank` dimensions (innermost first) with element type `type`; strides are in bytes
+// for dims 1..rank-1.  Out-of-range elements of a box read as zero.  Returns false when the driver
+// rejects the map.
+inline bool make_tensor_map(CUtensorMap* m, CUtensorMapDataType type, const void* base, int rank,
+                            const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                            CUtensorMapSwizzle sw) {
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc || rank < 1 || rank > 5) return false;
   cuuint64_t d[5], s[4];
@@ -38,9 +40,13 @@ inline bool make_tensor_map_bf16(CUtensorMap* m, const void* base, int rank, con
     e[i] = 1;
     if (i + 1 < rank) s[i] = strides_bytes[i];
   }
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void*>(base), d, s, b, e,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return enc(m, type, (cuuint32_t)rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool make_tensor_map_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                                 const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
+  return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, rank, dims, strides_bytes, box, sw);
 }
 
 }  // namespace mla

@@ -117,3 +117,27 @@ def make_prefill_inputs(cfg: MLAConfig, seed: Optional[int] = None) -> Dict[str,
     q = _normal(rng, (B, S, cfg.n_h, cfg.d_h + cfg.d_r))
     q[..., cfg.d_h:] = _rope_interleaved(q[..., cfg.d_h:], pos[None, :].expand(B, S), cfg.rope_base)
     return {"cfg": cfg, "w_kv_b": w, "q": q.to(dt), "c_kv": c_kv, "k_r": k_r, "scale": cfg.scale}
+
+
+def quantize_latent_fp8(c_kv: torch.Tensor, block: int = 128):
+    """FP8 latent cache of a bf16/fp32 latent cache [..., d_c]: one fp32 scale per row and
+    128-feature block (block max / 448, 1 for an all-zero block) and E4M3 codes of c / scale
+    (torch's float8_e4m3fn cast, round to nearest even).  Returns (c8 uint8 [..., d_c],
+    kv_scale float32 [..., d_c / block], c_deq bf16 [..., d_c]) where c_deq is the cache the kernel
+    reads back: bf16(float(code) * scale), one fp32 product then one rounding."""
+    x = c_kv.float()
+    shp = x.shape
+    blocks = x.reshape(*shp[:-1], shp[-1] // block, block)
+    scale = blocks.abs().amax(dim=-1) / 448.0
+    scale = torch.where(scale > 0, scale, torch.ones_like(scale)).to(torch.float32)
+    q = (blocks / scale[..., None]).reshape(shp).to(torch.float8_e4m3fn)
+    c8 = q.view(torch.uint8)
+    deq = (q.to(torch.float32).reshape(*shp[:-1], shp[-1] // block, block) * scale[..., None]).reshape(shp)
+    return c8, scale, deq.to(torch.bfloat16)
+
+
+def pack_fp8_cache(c8: torch.Tensor, kv_scale: torch.Tensor, k_r: torch.Tensor) -> torch.Tensor:
+    """One 656-byte row per cached token: 512 E4M3 codes, 4 fp32 scales, 64 bf16 rotary features."""
+    rows = torch.cat([c8.contiguous().view(torch.uint8), kv_scale.contiguous().view(torch.uint8),
+                      k_r.to(torch.bfloat16).contiguous().view(torch.uint8)], dim=-1)
+    return rows.contiguous()

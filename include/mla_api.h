@@ -148,6 +148,31 @@ mla_status mla_decode_absorb(mla_dims dims, mla_dtype dtype, int32_t B,
                              void* workspace, size_t ws_bytes, int32_t* dev_err, void* stream);
 
 /*
+ * mla_decode_absorb_fp8kv - mla_decode_absorb over an FP8 latent cache (dense, one token per
+ * sequence).  The latent rows are stored as FP8 E4M3 codes with one fp32 scale per 128 latent
+ * features of each row (the 128-wide blocks of the FP8 weights, "Key-value down-projection",
+ * linear excerpt, applied per cached token: a reading, the pages keep the cache in bf16); the
+ * rotary key stays bf16.  The kernel dequantises on chip, c_kv[t, f] = bf16(float(e4m3(c8[t, f])) *
+ * kv_scale[t, f / 128]) with one fp32 product and one round-to-nearest-even, and then computes
+ * exactly what mla_decode_absorb computes on that bf16 cache (bit-identical results).
+ *   c8        row t of sequence b: d_c codes at (uint8*)c8 + b*c8_bstride + t*c8_rstride (BYTES;
+ *             both multiples of 16)
+ *   kv_scale  row t of sequence b: d_c / 128 floats at kv_scale + b*sc_bstride + t*sc_rstride
+ *             (FLOATS; both multiples of 4)
+ *   k_r       bf16 rotary rows as in mla_decode_absorb
+ *   A packed 656-byte row [512 codes | 4 scales | 64 bf16 rotary features] is c8 = base,
+ *   kv_scale = base + 512, k_r = base + 528, row strides 656, 164 and 328.
+ *   Other arguments as in mla_decode_absorb (bf16 DeepSeek dimensions only; workspace as
+ *   mla_decode_workspace_size(dims, MLA_BF16, B, n_max, 0)).  Asynchronous on `stream`.
+ */
+mla_status mla_decode_absorb_fp8kv(mla_dims dims, int32_t B, const void* q_tilde, int64_t ldqt, const void* q_pe,
+                                   int64_t ldqp, const void* c8, int64_t c8_bstride, int64_t c8_rstride,
+                                   const float* kv_scale, int64_t sc_bstride, int64_t sc_rstride, const void* k_r,
+                                   int64_t kr_bstride, int64_t kr_rstride, int32_t n_max, const int32_t* lengths,
+                                   float scale, void* ctx_out, float* lse_out, void* workspace, size_t ws_bytes,
+                                   int32_t* dev_err, void* stream);
+
+/*
  * mla_decode_absorb_multi - mla_decode_absorb for T new tokens per sequence ("DeepSeek-V3.2-Exp -
  * Absorb key weights", decode excerpt: the queries are [batch, s, heads, features] with s = T, e.g.
  * speculative tokens).  The T tokens of sequence b are the last T of its lengths[b] cached rows;

@@ -9,16 +9,19 @@ Pinned against what the pages and the mathematics fix (see ``tests/test_oracle_p
 the absorb/naive identity, closed forms (one cached row, zero query, two keys),
 library special cases (``scaled_dot_product_attention`` in fp64), brute-force
 top-k masking, the page's parameter counts and cache-size formulas, the RMSNorm and
-rotation invariants of the cache append, and planted mistakes that must be caught.  Every function here has at least one such pin.
+rotation invariants of the cache append, the FP8 codes and block scales of the FP8 latent
+cache (``tests/test_oracle_fp8kv.py``), and planted mistakes that must be caught.  Every function here has at least one such pin.
 """
 
 from .mla_oracle import (  # noqa: F401
     absorb_q,
     absorbed_decode,
     cache_append,
+    e4m3_value,
     fp8_block_scale_shape,
     index_mask,
     latent_attention,
+    latent_cache_dequant,
     mha_cache_bytes,
     mla_cache_bytes,
     multi_token_decode,

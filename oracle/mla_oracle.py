@@ -341,3 +341,34 @@ def weight_dequant(w_q, scale, block: int = 128) -> np.ndarray:
     s = _f64(scale)
     assert s.shape == fp8_block_scale_shape(w.shape[0], w.shape[1], block), "scale grid shape"
     return w * s[np.arange(w.shape[0]) // block][:, np.arange(w.shape[1]) // block]
+
+
+# ----------------------------------------------------------------------------------------
+# FP8 latent cache (a reading: the weights' FP8 format applied to the cached latent rows)
+# ----------------------------------------------------------------------------------------
+
+def e4m3_value(code) -> np.ndarray:
+    """Value of FP8 E4M3 codes (uint8): sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
+    exponent field 0 holds the subnormals m/8 * 2^-6; the one all-ones pattern S.1111.111 is NaN
+    and there is no infinity (the finite "fn" variant the pages' float8 weights use, "Key-value
+    down-projection", linear excerpt).  Written out from that definition, code by code."""
+    c = np.asarray(code, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    val = sign * val
+    return np.where((c & 0x7F) == 0x7F, np.nan, val)
+
+
+def latent_cache_dequant(c8, kv_scale, block: int = 128) -> np.ndarray:
+    """The FP8 latent cache read back: c_kv[t, f] = e4m3(c8[t, f]) * kv_scale[t, f // block].  One
+    float32 scale per cached row and 128-feature block, the 128-wide blocks of the FP8 weights
+    ("Key-value down-projection", linear excerpt: one float32 scale per 128 x 128 block) applied to
+    each cached token's latent row, since rows are written one token at a time (a reading; the
+    pages keep the cache in bf16).  c8 [..., d_c] uint8 codes, kv_scale [..., d_c / block]."""
+    v = e4m3_value(c8)
+    s = _f64(kv_scale)
+    d_c = v.shape[-1]
+    assert s.shape[-1] == (d_c + block - 1) // block and s.shape[:-1] == v.shape[:-1], "scale grid shape"
+    return v * s[..., np.arange(d_c) // block]
