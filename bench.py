@@ -165,7 +165,7 @@ def run_reference(args, rank, world):
     print(json.dumps(line), flush=True)
 
 
-def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append", "fp8proj", "sparse_prefill",
+def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append", "fp8proj", "fp8kv", "sparse_prefill",
                                           "multi")):
     """The other workloads of the hot path, each timed on its own with CUDA events (L2 flushed
     before every launch): the ragged long-context decode, the V3.2 top-k decode, the naive causal
@@ -262,6 +262,35 @@ def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append
                                      "roofline_frac": max(nbytes / (peaks["hbm_gbs"] * 1e9),
                                                           flops / (peaks["bf16_tflops"] * 1e12)) / (ms * 1e-3)}
         del x, cache, c_kv, k_r, ws
+        torch.cuda.empty_cache()
+    if "fp8kv" in which:
+        # the decode workload over an FP8 latent cache: packed 656-byte rows (512 E4M3 codes, 4 fp32
+        # scales, 64 bf16 rotary features), dequantised on chip
+        from head_latent_attention_absorb_b200.inputs import pack_fp8_cache, quantize_latent_fp8
+        cfg = V3_DECODE
+        x = make_decode_inputs(cfg)
+        c8, sc, _ = quantize_latent_fp8(x["c_kv"])
+        rows = pack_fp8_cache(c8, sc, x["k_r"]).to(dev)
+        c8d, scd, krd = rows[..., :512], rows[..., 512:528].view(torch.float32), rows[..., 528:].view(torch.bfloat16)
+        qt = torch.from_numpy(np.random.default_rng(cfg.seed + 500).standard_normal(
+            (cfg.B, cfg.n_h, cfg.d_c), dtype=np.float32) * 0.2).to(torch.bfloat16).to(dev)
+        qp, lengths = x["q_pe"].to(dev), x["lengths"].to(dev)
+        ctx = torch.empty((cfg.B, cfg.n_h, cfg.d_c), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty((api.mla_decode_workspace_size(cfg.dims, torch.bfloat16, cfg.B, cfg.n_max),),
+                         dtype=torch.uint8, device=dev)
+        ms = timed(lambda: api.mla_decode_absorb_fp8kv(cfg.dims, qt, qp, c8d, scd, krd, lengths, cfg.scale, ctx=ctx,
+                                                       workspace=ws, stream=stream))
+        keys = int(x["lengths"].to(torch.int64).sum())
+        nbytes = keys * (cfg.d_c + 16 + cfg.d_r * 2) + cfg.B * cfg.n_h * (cfg.d_c + cfg.d_r + cfg.d_c) * 2
+        flops = 2 * keys * cfg.n_h * (2 * cfg.d_c + cfg.d_r)
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        tf = flops / (ms * 1e-3) / 1e12
+        out["fp8kv_b32_n4096"] = {"call": "mla_decode_absorb_fp8kv", "ms": ms, "tokens_per_s": cfg.B / (ms * 1e-3),
+                                  "algorithmic_bytes": nbytes, "achieved_GBs": gbs, "hbm_frac": gbs / peaks["hbm_gbs"],
+                                  "flops": flops, "tflops": tf, "tensor_frac": tf / peaks["bf16_tflops"],
+                                  "roofline_frac": max(nbytes / (peaks["hbm_gbs"] * 1e9),
+                                                       flops / (peaks["bf16_tflops"] * 1e12)) / (ms * 1e-3)}
+        del x, rows, ws
         torch.cuda.empty_cache()
     if "fp8proj" in which:
         # the two projections of the decode workload with an e4m3 wkv_b and 128 x 128 block scales
@@ -497,7 +526,7 @@ def main():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the timings of the secondary workloads (ragged, top-k, prefill, cache append, "
                          "FP8 projections, sparse prefill)")
-    ap.add_argument("--only", choices=["ragged", "sparse", "prefill", "append", "fp8proj", "sparse_prefill", "multi"],
+    ap.add_argument("--only", choices=["ragged", "sparse", "prefill", "append", "fp8proj", "fp8kv", "sparse_prefill", "multi"],
                     help="time only this secondary workload (--steps launches after 3 warm-up ones) and print "
                          "its entry; a small command for profilers, not a bench line")
     args = ap.parse_args()

@@ -383,6 +383,34 @@ __device__ __forceinline__ void gather_half(const Params& p, int row_of_lane, in
   cp_async_mbar_arrive(bar);
 }
 
+// FP8 latent cache: rows [r0, r1) of a raw tile (e4m3 latent half, 256 bytes per row, then the
+// rows' 4 fp32 scales) written as bf16 into a stage in exactly the layout the TMA boxes of the bf16
+// cache give: slab s, row r, 16-byte chunk c at s * 8 KB + 128 r + 16 (c ^ (r & 7)).  Lane l converts
+// chunk l (features 8 l .. 8 l + 7 of this CTA's half); value = bf16(float(code) * scale of its
+// 128-feature block), one fp32 product and one rounding.  The writes are made visible to the
+// tensor cores (async proxy) before returning.
+__device__ __forceinline__ void convert_fp8_rows(const uint8_t* raw, uint32_t stage, int r0, int r1, uint32_t rank,
+                                                 int lane) {
+  const int blk = 2 * (int)rank + (lane >> 4);
+  const uint32_t dst = stage + (uint32_t)(lane >> 3) * kSlabBytes, chunk = (uint32_t)(lane & 7);
+#pragma unroll 4
+  for (int r = r0; r < r1; ++r) {
+    const uint2 w = *reinterpret_cast<const uint2*>(raw + r * 256 + lane * 8);
+    const float sc = reinterpret_cast<const float*>(raw + kRawLatBytes + r * 16)[blk];
+    uint32_t o[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t word = j < 2 ? w.x : w.y;
+      const __half2_raw hr =
+          __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((word >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+      o[j] = pack_bf16x2(f.x * sc, f.y * sc);
+    }
+    st_shared_v4_b32(dst + r * 128 + ((chunk ^ (uint32_t)(r & 7)) << 4), o[0], o[1], o[2], o[3]);
+  }
+  fence_proxy_async_smem();
+}
+
 // Walks the segments (sequence, first tile, end tile) of this cluster's range.
 struct SegIter {
   int b, tb, t, hi, len0;
@@ -514,8 +542,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       // dense: the producer's arrive.expect_tx + the TMA bytes; sparse: one cp.async arrival per lane
       // of the two gathering warps
-      // FP8 cache: the producer's arrive.expect_tx for the rotary slab + the conversion warp's arrival
-      mbar_init(smem_u32(&sm.full[s]), kFp8 ? 2 : (p.topk > 0 ? 64 : 1));
+      // FP8 cache: the producer's arrive.expect_tx for the rotary slab + the two converting warps
+      mbar_init(smem_u32(&sm.full[s]), kFp8 ? 3 : (p.topk > 0 ? 64 : 1));
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     // softmax-side arrivals are one per softmax warp, after a __syncwarp
@@ -545,7 +573,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.mrg_full2[i]), 1);
       mbar_init(smem_u32(&sm.mrg_empty2[i]), kSoftmaxWarps);
       mbar_init(smem_u32(&sm.raw_full[i]), 1);
-      mbar_init(smem_u32(&sm.raw_empty[i]), 1);
+      mbar_init(smem_u32(&sm.raw_empty[i]), 2);  // the two converting warps
     }
     sm.abort = 0;
     fence_mbar_init();
@@ -586,6 +614,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool whole;
       uint32_t it = 0, nseg_p = 0;
       bool ok = true, q_issued = false;
+      // FP8 cache: the producer's half of tile t's conversion (its stage is already free: the loads
+      // of tile t waited for it)
+      auto convert_prev = [&](uint32_t t) -> bool {
+        const uint32_t rs = t & 1u;
+        const bool got = mbar_wait(smem_u32(&sm.raw_full[rs]), (t >> 1) & 1u, abort_flag, kWaitLimitNs);
+        if (!__all_sync(0xffffffffu, got)) {
+          if (lane == 0) fail_timeout(sm, p.err);
+          return false;
+        }
+        convert_fp8_rows(smem + kRawOff + rs * kRawSlotBytes, smem_u32(stages + (t % kNS) * kStageBytes), kTile / 2,
+                         kTile, rank, lane);
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(smem_u32(&sm.full[t % kNS]));
+          mbar_arrive(smem_u32(&sm.raw_empty[rs]));
+        }
+        return true;
+      };
       while (ok && seg.next(b, begin, end, len, whole, base)) {
         if (!q_issued) {
           griddep_wait();  // the absorbed query is the preceding kernel's output
@@ -643,6 +689,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
+            // rows [32, 64) of the previous tile (its loads were issued one tile ago)
+            if (it > 0 && !convert_prev(it - 1)) {
+              ok = false;
+              break;
+            }
           } else if (p.topk == 0) {
             if (lane == 0) {
               mbar_arrive_expect_tx(bar, kStageBytes);
@@ -696,6 +747,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         ++nseg_p;
       }
+      // FP8 cache: the last tile's rows [32, 64)
+      if (kFp8 && ok && it > 0 && !convert_prev(it - 1)) ok = false;
       // drain: every load issued must have landed before the CTA may exit
       if (lane == 0) {
         const uint32_t first = it > (uint32_t)kNS ? it - kNS : 0;
@@ -887,18 +940,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0) mbar_arrive(smem_u32(&sm.xch_drained));
   } else if (kFp8 && warp == kGatherWarp) {
     // ------------------------------------------------------------------ FP8 cache: conversion warp
-    // Every tile: wait for its raw slot (e4m3 latent half + scales) and for its stage, write the
-    // dequantised latent as bf16 into the stage in exactly the layout the TMA boxes of the bf16
-    // cache give (slab s, row r, 16-byte chunk c at s * 8 KB + 128 r + 16 (c ^ (r & 7))), then release
-    // both.  Value = e4m3 code * the row's fp32 scale of its 128-feature block, rounded to bf16.
-    // Lane l converts chunk l (features 8 l .. 8 l + 7 of this CTA's half) of every row.
+    // Every tile: wait for its raw slot (e4m3 latent half + scales) and for its stage, convert half
+    // of its rows into the stage, then count on both (the producer converts the other half).
     SegIter seg(sm, p);
     int b, begin, end, len, base;
     bool whole;
     uint32_t it = 0;
     bool ok = true;
-    const int blk = 2 * (int)rank + (lane >> 4);
-    const uint32_t out_off = (uint32_t)(lane >> 3) * kSlabBytes, chunk = (uint32_t)(lane & 7);
     while (ok && seg.next(b, begin, end, len, whole, base)) {
       for (int i = begin; i < end && ok; ++i, ++it) {
         const uint32_t st = it % kNS, rs = it & 1u;
@@ -909,24 +957,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        const uint8_t* raw = smem + kRawOff + rs * kRawSlotBytes;
-        const uint32_t dst = smem_u32(stages + st * kStageBytes) + out_off;
-#pragma unroll 4
-        for (int r = 0; r < kTile; ++r) {
-          const uint2 w = *reinterpret_cast<const uint2*>(raw + r * 256 + lane * 8);
-          const float sc = reinterpret_cast<const float*>(raw + kRawLatBytes + r * 16)[blk];
-          uint32_t o[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const uint32_t word = j < 2 ? w.x : w.y;
-            const __half2_raw hr =
-                __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)((word >> (16 * (j & 1))) & 0xffffu), __NV_E4M3);
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-            o[j] = pack_bf16x2(f.x * sc, f.y * sc);
-          }
-          st_shared_v4_b32(dst + r * 128 + ((chunk ^ (uint32_t)(r & 7)) << 4), o[0], o[1], o[2], o[3]);
-        }
-        fence_proxy_async_smem();  // the MMAs read the stage through the async proxy
+        // rows [0, 32); the producer converts rows [32, 64) one tile behind its loads
+        convert_fp8_rows(smem + kRawOff + rs * kRawSlotBytes, smem_u32(stages + st * kStageBytes), 0, kTile / 2, rank,
+                         lane);
         __syncwarp();
         if (lane == 0) {
           mbar_arrive(smem_u32(&sm.full[st]));
