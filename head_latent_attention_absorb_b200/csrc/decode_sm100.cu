@@ -614,24 +614,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       bool whole;
       uint32_t it = 0, nseg_p = 0;
       bool ok = true, q_issued = false;
-      // FP8 cache: the producer's half of tile t's conversion (its stage is already free: the loads
-      // of tile t waited for it)
-      auto convert_prev = [&](uint32_t t) -> bool {
-        const uint32_t rs = t & 1u;
-        const bool got = mbar_wait(smem_u32(&sm.raw_full[rs]), (t >> 1) & 1u, abort_flag, kWaitLimitNs);
-        if (!__all_sync(0xffffffffu, got)) {
-          if (lane == 0) fail_timeout(sm, p.err);
-          return false;
-        }
-        convert_fp8_rows(smem + kRawOff + rs * kRawSlotBytes, smem_u32(stages + (t % kNS) * kStageBytes), kTile / 2,
-                         kTile, rank, lane);
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(smem_u32(&sm.full[t % kNS]));
-          mbar_arrive(smem_u32(&sm.raw_empty[rs]));
-        }
-        return true;
-      };
       while (ok && seg.next(b, begin, end, len, whole, base)) {
         if (!q_issued) {
           griddep_wait();  // the absorbed query is the preceding kernel's output
@@ -689,11 +671,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            // rows [32, 64) of the previous tile (its loads were issued one tile ago)
-            if (it > 0 && !convert_prev(it - 1)) {
-              ok = false;
-              break;
-            }
           } else if (p.topk == 0) {
             if (lane == 0) {
               mbar_arrive_expect_tx(bar, kStageBytes);
@@ -747,8 +724,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         }
         ++nseg_p;
       }
-      // FP8 cache: the last tile's rows [32, 64)
-      if (kFp8 && ok && it > 0 && !convert_prev(it - 1)) ok = false;
       // drain: every load issued must have landed before the CTA may exit
       if (lane == 0) {
         const uint32_t first = it > (uint32_t)kNS ? it - kNS : 0;
@@ -833,6 +808,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
     };
+    // FP8 cache: the P*V warp converts rows [32, 64) of every tile (the conversion warp rows
+    // [0, 32)), two tiles ahead of the tile whose P it waits for next: tiles 0 and 1 before the
+    // first P*V, tile t + 2 right after issuing P*V(t)
+    const uint32_t ntiles_fp8 = sm.hi > sm.lo ? (uint32_t)(sm.hi - sm.lo) : 0u;
+    auto convert_half = [&](uint32_t t) -> bool {
+      const uint32_t st = t % kNS, rs = t & 1u;
+      if (!wait_or_fail(smem_u32(&sm.raw_full[rs]), (t >> 1) & 1u, false)) return false;
+      if (!wait_or_fail(smem_u32(&sm.empty[st]), ((t / kNS) & 1u) ^ 1u, false)) return false;
+      convert_fp8_rows(smem + kRawOff + rs * kRawSlotBytes, smem_u32(stages + st * kStageBytes), kTile / 2, kTile, rank,
+                       lane);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(smem_u32(&sm.full[st]));
+        mbar_arrive(smem_u32(&sm.raw_empty[rs]));
+      }
+      return true;
+    };
+    if (kFp8 && !is_qk)
+      for (uint32_t t = 0; t < 2 && t < ntiles_fp8 && ok; ++t) ok = convert_half(t);
     // O += P(t) V(t) over this CTA's 256 latent features
     auto issue_pv = [&](uint32_t t, bool first_of_seg) {
       if (!wait_or_fail(smem_u32(&sm.p_full), t & 1u, false)) return;
@@ -857,7 +851,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int i = begin; i < end && ok; ++i) issue_qk(it++, i);
       } else {
-        for (int i = begin; i < end && ok; ++i) issue_pv(it++, i == begin);
+        for (int i = begin; i < end && ok; ++i) {
+          issue_pv(it++, i == begin);
+          // FP8 cache: rows [32, 64) of the tile two ahead, while this warp would wait for P
+          if (kFp8 && ok && it + 1 < ntiles_fp8) ok = convert_half(it + 1);
+        }
       }
       ++nseg;
     }
@@ -941,7 +939,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   } else if (kFp8 && warp == kGatherWarp) {
     // ------------------------------------------------------------------ FP8 cache: conversion warp
     // Every tile: wait for its raw slot (e4m3 latent half + scales) and for its stage, convert half
-    // of its rows into the stage, then count on both (the producer converts the other half).
+    // of its rows into the stage, then count on both (the P*V warp converts the other half).
     SegIter seg(sm, p);
     int b, begin, end, len, base;
     bool whole;
@@ -957,7 +955,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        // rows [0, 32); the producer converts rows [32, 64) one tile behind its loads
+        // rows [0, 32); the P*V warp converts rows [32, 64) two tiles ahead
         convert_fp8_rows(smem + kRawOff + rs * kRawSlotBytes, smem_u32(stages + st * kStageBytes), 0, kTile / 2, rank,
                          lane);
         __syncwarp();
