@@ -37,7 +37,7 @@ L2_FLUSH_BYTES = 256 << 20
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one decode launch on this workload,
 # from one ncu capture of the decode kernel, valid only for the kernel source it was taken on
 # (sha256 prefix of csrc/decode_sm100.cu).
-DECODE_TRAFFIC = {"bytes": 155_855_104 + 3_634_944, "source_sha256": "e288f1f5373cecdb"}
+DECODE_TRAFFIC = {"bytes": 155_889_152 + 3_018_496, "source_sha256": "1e2e3f810ae0b3b4"}
 
 
 def decode_traffic():

@@ -15,19 +15,27 @@
 //   swizzled rotary slab) into a 4-stage ring; S = Q K^T runs with Q held in TMEM (A operand)
 //   and K in shared memory; P (bf16) is written to TMEM and O += P V reads V from the SAME
 //   shared-memory tile (K-major for the scores, MN-major for the values).
+// * Top-k decode: the tile's selected rows are gathered with per-lane cp.async into the layout the
+//   TMA boxes would give, keys 0..31 by the producer and keys 32..63 by warp 15.
+// * FP8 latent cache (decode_kernel<true>): E4M3 rows and per-128-feature fp32 scales land in two
+//   raw slots behind a 3-stage bf16 ring; warp 15 and the P.V warp convert them into the stages'
+//   bf16 layout on chip, and the rest of the kernel is unchanged.
 // * Warp roles: warp 0 = TMA producer; warp 1 = TMEM allocator + score-MMA issuer; warp 2 =
-//   P.V-MMA issuer; warps 3..6 = exchange (read S from TMEM, round to fp16, stage, bulk-copy to
-//   the peer); warps 7..14 = softmax (two per TMEM lane quadrant, 32 keys each, agreeing on the
-//   row maximum through shared memory), O rescale and epilogue.
+//   P.V-MMA issuer (and, with the FP8 cache, converter of half of every tile); warps 3..6 =
+//   exchange (read S from TMEM, round to fp16, stage, bulk-copy to the peer); warps 7..14 =
+//   softmax (two per TMEM lane quadrant, 32 keys each, agreeing on the row maximum through shared
+//   memory), O rescale and epilogue; warp 15 = second gatherer (top-k) or converter (FP8 cache).
+//   512 threads x 128 registers fill the register file.
 // * Online softmax in base 2 with the scale folded in; the running maximum is only raised (and
 //   O rescaled in TMEM) when it grows by more than 8, so rescales are rare.
 // * Work split: when every non-empty sequence can get its own clusters, each sequence is cut into
 //   chunks of at most `chunk` tiles and cluster i takes chunk i (one sequence per cluster, so the
 //   query is loaded once, by TMA, and no pipeline restart happens mid-kernel); otherwise the
 //   concatenated tiles of all sequences are cut into equal contiguous ranges.  A cluster that
-//   covers a whole sequence writes ctx directly; the others write fp32 partials (O, m, l) and the
-//   last cluster to finish a sequence (an arrival counter per sequence and latent half) merges
-//   them, so no second kernel is launched.
+//   covers a whole sequence writes ctx directly; the others write bf16 partials (O normalised,
+//   with its m and l) and the last cluster to finish a sequence (an arrival counter per sequence
+//   and latent half, counted by the producer at the segment's last tile) merges two of them;
+//   three or more are merged in head slices by all the sequence's clusters.  No second kernel.
 // * Every wait is a bounded mbarrier wait (global timer); on expiry the kernel records
 //   MLA_ERR_TIMEOUT, drains and returns.
 #include <cuda.h>
@@ -142,6 +150,8 @@ struct Smem {
   long long total;       // tiles of all sequences
   int bad;               // some length outside [1, n_max]
   int nslots, is_last;
+  int q_seg;             // segments whose query the softmax warps have copied (so whose predecessor's
+                         // epilogue is done with the slot list): a count, free of phase aliasing
 };
 
 __device__ __forceinline__ int clamp_len(int len, int n_max) { return len < 0 ? 0 : (len > n_max ? n_max : len); }
@@ -576,6 +586,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&sm.raw_empty[i]), 2);  // the two converting warps
     }
     sm.abort = 0;
+    sm.q_seg = 0;
     fence_mbar_init();
     prefetch_tensormap(&p.tm_ckv);
     prefetch_tensormap(&p.tm_kr);
@@ -702,7 +713,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             // epilogue is done with the slot list.
             int okq = 1;
             if (lane == 0) {
-              if (nseg_p > 0 && !mbar_wait(smem_u32(&sm.q_full), nseg_p & 1u, abort_flag, kWaitLimitNs)) okq = 0;
+              if (nseg_p > 0) {
+                // (a count, not q_full's phase parity: after short whole segments the producer can be
+                // two segments ahead, and a parity wait would pass on an older phase)
+                const uint64_t t0 = globaltimer();
+                while (*reinterpret_cast<volatile int*>(&sm.q_seg) < (int)nseg_p + 1) {
+                  if (*abort_flag || globaltimer() - t0 > kWaitLimitNs) {
+                    okq = 0;
+                    break;
+                  }
+                  __nanosleep(32);
+                }
+                __threadfence_block();
+              }
               if (okq) {
                 const int ns = list_slots(p, sm, base, tiles_of(len));
                 // up to p.slice_above partials (kMergeLastMax = 2 when the whole grid is resident,
@@ -1104,6 +1127,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           if (mbar_wait(smem_u32(&sm.q_full), 0, abort_flag, kWaitLimitNs)) {
             mbar_arrive_remote(x_free_peer0);
             mbar_arrive_remote(x_free_peer0 + 8);
+            __threadfence_block();
+            *reinterpret_cast<volatile int*>(&sm.q_seg) = 1;
           } else {
             fail_timeout(sm, p.err);
           }
@@ -1134,6 +1159,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         warp_arrive(smem_u32(&sm.q_full));
+        if (sw == 0 && lane == 0) {
+          // every softmax warp has finished the previous segment and copied this one's query
+          if (mbar_wait(smem_u32(&sm.q_full), nseg & 1u, abort_flag, kWaitLimitNs)) {
+            __threadfence_block();
+            *reinterpret_cast<volatile int*>(&sm.q_seg) = (int)nseg + 1;
+          } else {
+            fail_timeout(sm, p.err);
+          }
+        }
       }
       float m_run = -INFINITY, l_run = 0.f;
       for (int i = begin; i < end && ok; ++i) {

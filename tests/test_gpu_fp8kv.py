@@ -103,3 +103,23 @@ def test_fp8kv_bad_length_and_host_checks(dev):
     with pytest.raises(RuntimeError):
         api.mla_decode_absorb_fp8kv(cfg.dims, qt.to(dev), x["q_pe"].to(dev), c8d, sc.to(dev),
                                     x["k_r"].contiguous().to(dev), x["lengths"].to(dev), cfg.scale)
+
+
+def test_fp8kv_many_sequences_range_plan(dev):
+    """B = 100 sequences of 1..300 rows: more sequences than clusters, so the work plan cuts the
+    concatenated tiles into ranges and a cluster walks several sequences.  The conversion runs on a
+    tile counter that carries over the segments; bit-equal to the bf16 decode as above."""
+    B = 100
+    lengths = torch.from_numpy(np.random.default_rng(100).integers(1, 301, size=B).astype(np.int32))
+    cfg = V3_DECODE.with_(B=B, n_max=300)
+    x, c8, sc, deq, qt = _case(cfg, lengths=lengths)
+    ctx8, lse8, e = _fp8_call(cfg, dev, qt, x["q_pe"], c8, sc, x["k_r"], lengths, packed=True)
+    assert e == 0
+    lse = torch.empty_like(lse8)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    ctx = api.mla_decode_absorb(cfg.dims, qt.to(dev), x["q_pe"].to(dev), deq.to(dev), x["k_r"].contiguous().to(dev),
+                                lengths.to(dev), cfg.scale, lse=lse, dev_err=err)
+    torch.cuda.synchronize()
+    assert api.mla_get_device_error(err) == 0
+    assert torch.equal(ctx8, ctx)
+    assert torch.equal(lse8, lse)

@@ -254,6 +254,55 @@ def test_topk_full_set_equals_dense_and_order_free(dev):
     check_close(rev, to_np(sp), torch.bfloat16, "top-k reversed order")
 
 
+def test_topk_many_sequences_range_plan(dev):
+    """B = 100 sequences of 200 rows with every position selected, in order: more sequences than
+    clusters, so both gathering warps walk several sequences per cluster.  Same result as the dense
+    decode, and the oracle on three sequences."""
+    B, L = 100, 200
+    cfg = SPARSE_V32.with_(B=B, n_max=L, topk=L)
+    x = upload(make_decode_inputs(cfg, lengths=torch.full((B,), L, dtype=torch.int32)), dev)
+    qt = torch.from_numpy(oracle_qt(x)).to(torch.bfloat16).cuda()
+    tk = torch.arange(L, dtype=torch.int32).repeat(B, 1).contiguous().cuda()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    sp = api.mla_decode_absorb(cfg.dims, qt, x["q_pe_d"], x["c_kv_d"], x["k_r_d"], x["len_d"], cfg.scale,
+                               topk_idx=tk, dev_err=err)
+    dense = api.mla_decode_absorb(cfg.dims, qt, x["q_pe_d"], x["c_kv_d"], x["k_r_d"], x["len_d"], cfg.scale)
+    torch.cuda.synchronize()
+    assert api.mla_get_device_error(err) == 0
+    check_close(sp, to_np(dense), torch.bfloat16, "top-k every position vs dense, B=100")
+    for b in (0, 57, B - 1):
+        want, _, _ = O.latent_attention(qt[b].cpu(), x["q_pe"][b], x["c_kv"][b, :L], x["k_r"][b, :L], cfg.scale,
+                                        np.arange(L))
+        check_close(sp[b], want, torch.bfloat16, f"top-k range plan b={b}")
+
+
+def test_dense_many_sequences_range_plan(dev):
+    """B = 100 sequences of 1..300 rows: a cluster's range crosses many sequences, short ones whole
+    and the ones at its ends split with a neighbour cluster, so split-KV arrivals of consecutive
+    segments follow each other closely.  Against the oracle on every sequence's first head row and
+    in full on four sequences (the shortest, the longest, two split ones)."""
+    B = 100
+    lengths = torch.from_numpy(np.random.default_rng(101).integers(1, 301, size=B).astype(np.int32))
+    cfg = V3_DECODE.with_(B=B, n_max=300)
+    x = upload(make_decode_inputs(cfg, lengths=lengths), dev)
+    qt = torch.from_numpy(oracle_qt(x)).to(torch.bfloat16)
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    lse = torch.empty((B, cfg.n_h), dtype=torch.float32, device="cuda")
+    ctx = api.mla_decode_absorb(cfg.dims, qt.cuda(), x["q_pe_d"], x["c_kv_d"], x["k_r_d"], x["len_d"], cfg.scale,
+                                lse=lse, dev_err=err)
+    torch.cuda.synchronize()
+    assert api.mla_get_device_error(err) == 0
+    Ls = lengths.numpy()
+    full = {int(np.argmin(Ls)), int(np.argmax(Ls)), 37, 62}
+    for b in range(B):
+        L = int(Ls[b])
+        heads = slice(None) if b in full else slice(0, 1)
+        want_ctx, want_lse, _ = O.latent_attention(qt[b, heads], x["q_pe"][b, heads], x["c_kv"][b, :L],
+                                                   x["k_r"][b, :L], cfg.scale)
+        check_close(ctx[b, heads], want_ctx, torch.bfloat16, f"ctx b={b} L={L}")
+        check_close(lse[b, heads], want_lse, torch.bfloat16, f"lse b={b} L={L}")
+
+
 # ------------------------------------------------------------------------------------------
 # Naive causal prefill, B=2, S=2048
 # ------------------------------------------------------------------------------------------
