@@ -1,9 +1,8 @@
 """mla_decode_absorb_static: the decode entry point for callers that cannot allocate device memory
 (it uses the library's built-in scratch instead of a caller workspace).  Checked through the C ABI
-against mla_decode_absorb with a caller workspace, on consecutive calls that reuse the scratch.
-
-This file is collected last on purpose, so that a run stopping at the first failure has run every
-other test before it; it also passes when run on its own in a fresh process."""
+against mla_decode_absorb with a caller workspace, on consecutive calls that reuse the scratch and on
+replays of a CUDA graph that captured the call.  It also passes when run on its own in a fresh
+process."""
 
 import pytest
 import torch
@@ -69,3 +68,37 @@ def test_static_scratch_rejects_other_paths(dev):
     with pytest.raises(MLAError, match="UNSUPPORTED"):
         api.mla_decode_absorb_static(cfg.dims, t["qt"].float(), t["qp"].float(), t["c"].float(), t["k"].float(),
                                      t["lens"], cfg.scale)
+
+
+def test_static_scratch_in_a_cuda_graph(dev):
+    """The use the entry point is for: a warm call (it looks up the scratch), then the call captured
+    in a CUDA graph and replayed twice.  B = 4 with split sequences, so every replay publishes and
+    merges partials in the shared scratch with the same launch tag; both replays equal the
+    workspace decode bit for bit."""
+    B, n_max, lengths = CASES[0]
+    cfg, t = _case(B, n_max, lengths)
+    lse_ref = torch.empty((B, 128), dtype=torch.float32, device=dev)
+    ref = api.mla_decode_absorb(cfg.dims, t["qt"], t["qp"], t["c"], t["k"], t["lens"], cfg.scale, lse=lse_ref)
+    ctx = torch.empty((B, 128, 512), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, 128), dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    api.mla_decode_absorb_static(cfg.dims, t["qt"], t["qp"], t["c"], t["k"], t["lens"], cfg.scale,
+                                 ctx=ctx, lse=lse, dev_err=err)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(cap):
+        with torch.cuda.graph(graph, stream=cap):
+            api.mla_decode_absorb_static(cfg.dims, t["qt"], t["qp"], t["c"], t["k"], t["lens"], cfg.scale,
+                                         ctx=ctx, lse=lse, dev_err=err)
+    torch.cuda.synchronize()
+    for rep in range(2):
+        ctx.fill_(float("nan"))
+        lse.fill_(float("nan"))
+        graph.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(ctx, ref), f"ctx replay {rep}"
+        assert torch.equal(lse, lse_ref), f"lse replay {rep}"
+    assert api.mla_get_device_error(err) == 0
+    del graph

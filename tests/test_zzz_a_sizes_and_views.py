@@ -79,7 +79,7 @@ def test_query_as_views_of_one_tensor(v3):
 MLA_ERR_INDEX, MLA_ERR_LENGTH = 4, 7
 
 
-def host_verdict(idx: np.ndarray, lengths, n_max: int) -> int:
+def host_index_status(idx: np.ndarray, lengths, n_max: int) -> int:
     """What the flag must hold: 0, or the first error class a scan of the rows finds (the kernel
     raises every error it sees, the first to land wins, so the test cases carry one class each)."""
     for b, row in enumerate(idx):
@@ -91,7 +91,7 @@ def host_verdict(idx: np.ndarray, lengths, n_max: int) -> int:
     return 0
 
 
-def device_verdict(idx: np.ndarray, lengths, n_max: int) -> int:
+def device_index_status(idx: np.ndarray, lengths, n_max: int) -> int:
     t = torch.from_numpy(np.ascontiguousarray(idx, dtype=np.int32)).cuda()
     ln = None if lengths is None else torch.as_tensor(np.asarray(lengths, dtype=np.int32)).cuda()
     err = api.mla_check_topk(t, n_max, ln)
@@ -102,8 +102,8 @@ def test_sparse_workload_indices_are_valid(dev):
     cfg = SPARSE_V32
     x = make_decode_inputs(cfg)
     idx, lengths = x["topk"].numpy(), x["lengths"].numpy()
-    assert host_verdict(idx, lengths, cfg.n_max) == 0
-    assert device_verdict(idx, lengths, cfg.n_max) == 0
+    assert host_index_status(idx, lengths, cfg.n_max) == 0
+    assert device_index_status(idx, lengths, cfg.n_max) == 0
 
 
 @pytest.mark.parametrize("case", ["duplicate", "too_large", "negative", "zero_length", "no_lengths_ok"])
@@ -122,10 +122,10 @@ def test_each_error_class(dev, case):
         lengths[2] = 0
     elif case == "no_lengths_ok":
         lengths = None
-    want = host_verdict(idx, lengths, n_max)
+    want = host_index_status(idx, lengths, n_max)
     assert want == {"duplicate": MLA_ERR_INDEX, "too_large": MLA_ERR_INDEX, "negative": MLA_ERR_INDEX,
                     "zero_length": MLA_ERR_LENGTH, "no_lengths_ok": 0}[case]
-    assert device_verdict(idx, lengths, n_max) == want
+    assert device_index_status(idx, lengths, n_max) == want
 
 
 def test_long_cache_bitmap(dev):
@@ -133,6 +133,6 @@ def test_long_cache_bitmap(dev):
     rng = np.random.default_rng(9)
     n_max, k = 1_000_000, 2048
     idx = np.stack([rng.choice(n_max, k, replace=False) for _ in range(3)])
-    assert device_verdict(idx, None, n_max) == 0
+    assert device_index_status(idx, None, n_max) == 0
     idx[2, 1000] = idx[2, 5]
-    assert device_verdict(idx, None, n_max) == MLA_ERR_INDEX
+    assert device_index_status(idx, None, n_max) == MLA_ERR_INDEX
