@@ -132,3 +132,66 @@ def test_host_validation_codes(L):
     assert L.mla_clear_device_error(None, None) == 1
     out = ctypes.c_int32(0)
     assert L.mla_get_device_error(None, ctypes.byref(out)) == 1
+
+
+def test_host_validation_codes_newer_entry_points(L):
+    """The FP8-cache decode, the multi-token decode, the static-scratch decode and the wait self-test
+    refuse bad arguments on the host (before any launch)."""
+    tiny = _capi.MLADims(4, 64, 16, 32, 32)
+
+    def fp8(**kw):
+        a = dict(dims=DS, B=2, qt=FAKE, ldqt=512, qp=FAKE, ldqp=64, c8=FAKE, c8b=4096 * 656, c8r=656,
+                 sc=FAKE, scb=4096 * 164, scr=164, kr=FAKE, krb=4096 * 328, krr=328, n_max=4096, lengths=FAKE,
+                 scale=0.07, ctx=FAKE, lse=None, ws=FAKE, wsb=1 << 40, err=None)
+        a.update(kw)
+        return L.mla_decode_absorb_fp8kv(*a.values(), None)
+
+    assert fp8(dims=tiny) == 2              # bf16 DeepSeek dimensions only
+    assert fp8(B=0) == 1
+    assert fp8(n_max=0) == 1
+    assert fp8(sc=None) == 1                # no scales
+    assert fp8(lengths=None) == 1
+    assert fp8(c8r=520) == 1                # code rows not a multiple of 16 bytes
+    assert fp8(c8b=4096 * 656 + 8) == 1     # batch stride not a multiple of 16 bytes
+    assert fp8(c8r=500) == 1                # narrower than d_c codes
+    assert fp8(scr=3) == 1                  # fewer than d_c / 128 scales per row
+    assert fp8(scr=166) == 1                # scale rows not a multiple of 4 floats
+    assert fp8(krr=330) == 1                # rotary rows not a multiple of 8 elements
+    assert fp8(ldqt=256) == 1
+    assert fp8(scale=0.0) == 1
+    assert fp8(scale=float("nan")) == 1
+    assert fp8(c8=FAKE + 8) == 1            # misaligned code rows
+    assert fp8(ws=None) == 6
+    assert fp8(wsb=16) == 6
+    assert fp8(ws=FAKE + 8) == 1            # misaligned workspace
+
+    def multi(**kw):
+        a = dict(dims=DS, dt=_capi.MLA_BF16, B=2, T=2, qt=FAKE, ldqt=512, qp=FAKE, ldqp=64, ckv=FAKE,
+                 cb=4096 * 576, cr=576, kr=FAKE, kb=4096 * 576, krr=576, n_max=4096, lengths=FAKE, scale=0.07,
+                 ctx=FAKE, lse=None, ws=FAKE, wsb=1 << 40, err=None)
+        a.update(kw)
+        return L.mla_decode_absorb_multi(*a.values(), None)
+
+    assert multi(dt=_capi.MLA_F32) == 2     # several tokens per sequence: bf16 only
+    assert multi(T=0) == 1
+    assert multi(T=4097) == 1               # more new tokens than cache rows
+    assert multi(B=0) == 1
+    assert multi(qt=None) == 1
+    assert multi(cr=577) == 1
+    assert multi(scale=-1.0) == 1
+    assert multi(ws=None) == 6
+    assert multi(T=1, ws=None) == 6         # T = 1 is the one-token decode and validates as such
+
+    def static(**kw):
+        a = dict(dims=DS, dt=_capi.MLA_BF16, B=2, qt=FAKE, ldqt=512, qp=FAKE, ldqp=64, ckv=FAKE,
+                 cb=4096 * 576, cr=576, kr=FAKE, kb=4096 * 576, krr=576, n_max=4096, lengths=FAKE, scale=0.07,
+                 ctx=FAKE, lse=None, err=None)
+        a.update(kw)
+        return L.mla_decode_absorb_static(*a.values(), None)
+
+    assert static(dt=_capi.MLA_F32) == 2
+    assert static(B=0) == 1
+    assert static(B=100_000, n_max=65536) == 6   # more split-KV scratch than the built-in array holds
+    assert L.mla_selftest_wait_timeout(1_000_000, None, None) == 1
+    assert L.mla_selftest_wait_timeout(10, FAKE, None) == 1            # below 1 us
+    assert L.mla_selftest_wait_timeout(2_000_000_000, FAKE, None) == 1  # above 1 s
