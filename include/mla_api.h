@@ -102,7 +102,9 @@ size_t mla_decode_workspace_size(mla_dims dims, mla_dtype dtype, int32_t B, int3
 
 /*
  * mla_decode_num_launches - how many kernels one mla_decode_absorb call with these sizes
- * launches on the current device (the split-KV plan decides whether a combine pass runs).
+ * launches on the current device: 1 for bf16 (partials merged inside the kernel); for fp32 the
+ * split-KV plan decides whether a combine pass runs.  (A bf16 top-k call over a cache whose batch
+ * stride is not n_max rows runs the CUDA-core path, which this count does not cover.)
  * 0 for arguments mla_decode_absorb would reject.
  */
 int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32_t n_max, int32_t topk);
@@ -130,6 +132,12 @@ int32_t mla_decode_num_launches(mla_dims dims, mla_dtype dtype, int32_t B, int32
  *            contents need no initialisation and are garbage afterwards
  *   dev_err  NULL or a device int32 flag; MLA_ERR_LENGTH / MLA_ERR_INDEX are stored there
  * Asynchronous on `stream`.
+ * Accuracy (bf16): the two CTAs of a pair each compute half of every score (288 of the 576
+ *   features, before the scale) and exchange it as fp16: a half-score beyond +-65504 saturates, and
+ *   each is rounded to 2^-11 of its magnitude, an error of about |half-score| * scale * 2^-11 in the
+ *   exponent of its softmax weight.  At DeepSeek magnitudes (RMS-normalised latent rows, scores of
+ *   a few tens) that is ~1e-3 relative, inside bf16; half-scores of several hundred exceed it.
+ *   The fp32 path and mla_decode_absorb_multi keep the scores in fp32.
  * Residency: the kernel is one persistent wave of CTA pairs sized by the occupancy query.  When a
  *   sequence is split into more than two pieces, every cluster holding a piece waits for all the
  *   others (the sliced merge), which needs every cluster resident at once.  The launcher uses that
