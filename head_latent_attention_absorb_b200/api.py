@@ -22,10 +22,14 @@ def dims_of(n_h: int, d_c: int, d_r: int, d_h: int, d_v: int) -> MLADims:
     return MLADims(n_h, d_c, d_r, d_h, d_v)
 
 
+def _dtc(dtype: torch.dtype) -> int:
+    if dtype not in _DT:
+        raise TypeError(f"unsupported dtype {dtype}")
+    return _DT[dtype]
+
+
 def _dt(t: torch.Tensor) -> int:
-    if t.dtype not in _DT:
-        raise TypeError(f"unsupported dtype {t.dtype}")
-    return _DT[t.dtype]
+    return _dtc(t.dtype)
 
 
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
@@ -72,11 +76,11 @@ def mla_absorb_q(dims, q_nope: torch.Tensor, w_kv_b: torch.Tensor, q_tilde: Opti
 
 
 def mla_decode_workspace_size(dims, dtype: torch.dtype, B: int, n_max: int, topk: int = 0) -> int:
-    return int(lib().mla_decode_workspace_size(_dims(dims), _DT[dtype], B, n_max, topk))
+    return int(lib().mla_decode_workspace_size(_dims(dims), _dtc(dtype), B, n_max, topk))
 
 
 def mla_decode_num_launches(dims, dtype: torch.dtype, B: int, n_max: int, topk: int = 0) -> int:
-    return int(lib().mla_decode_num_launches(_dims(dims), _DT[dtype], B, n_max, topk))
+    return int(lib().mla_decode_num_launches(_dims(dims), _dtc(dtype), B, n_max, topk))
 
 
 def mla_decode_absorb(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_kv: torch.Tensor, k_r: torch.Tensor,
@@ -244,7 +248,7 @@ def mla_out_up_fp8(dims, ctx: torch.Tensor, w_fp8: torch.Tensor, w_scale: torch.
 
 
 def mla_prefill_workspace_size(dims, dtype: torch.dtype, B: int, S: int) -> int:
-    return int(lib().mla_prefill_workspace_size(_dims(dims), _DT[dtype], B, S))
+    return int(lib().mla_prefill_workspace_size(_dims(dims), _dtc(dtype), B, S))
 
 
 def mla_prefill_naive(dims, q: torch.Tensor, c_kv: torch.Tensor, k_r: torch.Tensor, w_kv_b: torch.Tensor,

@@ -45,7 +45,7 @@ def test_shard_range_partitions():
 
 def test_two_gloo_ranks_shard_and_reduce():
     world, port = 2, _free_port()
-    out = mp.Manager().dict()
+    out = mp.get_context("spawn").Manager().dict()
     mp.start_processes(_worker, args=(world, port, out), nprocs=world, start_method="spawn", join=True)
     assert out[0][:2] == (0, 34) and out[1][:2] == (34, 33)
     for r in range(world):
