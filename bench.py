@@ -269,7 +269,7 @@ def time_secondary(dev, reps: int, which=("ragged", "sparse", "prefill", "append
         from head_latent_attention_absorb_b200.inputs import pack_fp8_cache, quantize_latent_fp8
         cfg = V3_DECODE
         x = make_decode_inputs(cfg)
-        c8, sc, _ = quantize_latent_fp8(x["c_kv"])
+        c8, sc = quantize_latent_fp8(x["c_kv"])
         rows = pack_fp8_cache(c8, sc, x["k_r"]).to(dev)
         c8d, scd, krd = rows[..., :512], rows[..., 512:528].view(torch.float32), rows[..., 528:].view(torch.bfloat16)
         qt = torch.from_numpy(np.random.default_rng(cfg.seed + 500).standard_normal(

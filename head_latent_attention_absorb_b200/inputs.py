@@ -120,20 +120,17 @@ def make_prefill_inputs(cfg: MLAConfig, seed: Optional[int] = None) -> Dict[str,
 
 
 def quantize_latent_fp8(c_kv: torch.Tensor, block: int = 128):
-    """FP8 latent cache of a bf16/fp32 latent cache [..., d_c]: one fp32 scale per row and
+    """Encodes a bf16/fp32 latent cache [..., d_c] as an FP8 cache: one fp32 scale per row and
     128-feature block (block max / 448, 1 for an all-zero block) and E4M3 codes of c / scale
     (torch's float8_e4m3fn cast, round to nearest even).  Returns (c8 uint8 [..., d_c],
-    kv_scale float32 [..., d_c / block], c_deq bf16 [..., d_c]) where c_deq is the cache the kernel
-    reads back: bf16(float(code) * scale), one fp32 product then one rounding."""
+    kv_scale float32 [..., d_c / block])."""
     x = c_kv.float()
     shp = x.shape
     blocks = x.reshape(*shp[:-1], shp[-1] // block, block)
     scale = blocks.abs().amax(dim=-1) / 448.0
     scale = torch.where(scale > 0, scale, torch.ones_like(scale)).to(torch.float32)
-    q = (blocks / scale[..., None]).reshape(shp).to(torch.float8_e4m3fn)
-    c8 = q.view(torch.uint8)
-    deq = (q.to(torch.float32).reshape(*shp[:-1], shp[-1] // block, block) * scale[..., None]).reshape(shp)
-    return c8, scale, deq.to(torch.bfloat16)
+    c8 = (blocks / scale[..., None]).reshape(shp).to(torch.float8_e4m3fn).view(torch.uint8)
+    return c8, scale
 
 
 def pack_fp8_cache(c8: torch.Tensor, kv_scale: torch.Tensor, k_r: torch.Tensor) -> torch.Tensor:

@@ -29,9 +29,18 @@ def dev():
     return torch.device("cuda:0")
 
 
+def kernel_read_back(c8: torch.Tensor, sc: torch.Tensor, block: int = 128) -> torch.Tensor:
+    """The bf16 cache the FP8-cache kernel reads back: bf16(float(code) * scale), one fp32 product
+    and one rounding (the oracle's latent_cache_dequant rounds once from the exact product instead)."""
+    shp = c8.shape
+    f = c8.view(torch.float8_e4m3fn).to(torch.float32).reshape(*shp[:-1], shp[-1] // block, block)
+    return (f * sc[..., None]).reshape(shp).to(torch.bfloat16)
+
+
 def _case(cfg, lengths=None, seed_q=11):
     x = make_decode_inputs(cfg, lengths=lengths)
-    c8, sc, deq = quantize_latent_fp8(x["c_kv"])
+    c8, sc = quantize_latent_fp8(x["c_kv"])
+    deq = kernel_read_back(c8, sc)
     qt = torch.from_numpy(O.absorb_q(x["q_nope"], x["w_kv_b"], cfg.n_h, cfg.d_h, cfg.d_v)).to(torch.bfloat16)
     return x, c8, sc, deq, qt
 
