@@ -678,6 +678,13 @@ __global__ void __launch_bounds__(32) sparse_lists_kernel(const int32_t* __restr
     if (on) list[count + __popc(m & ((1u << lane) - 1u))] = kt;
     count += __popc(m);
   }
+  // a query tile none of whose rows selected a visible key still runs one key tile, its diagonal,
+  // with every score masked: its rows end as empty rows (zeros, flagged), and every role of the
+  // attention kernel sees at least one key tile per query tile
+  if (count == 0) {
+    if (lane == 0) list[0] = qt;
+    count = 1;
+  }
   if (lane == 0) tile_count[b * n_qt + qt] = count;
 }
 static_assert(AT_BAROFF + sizeof(AttnBars) + 1024 <= 232448, "dynamic shared memory above the 227 KB per-CTA limit");
