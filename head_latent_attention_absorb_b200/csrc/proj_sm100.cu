@@ -4,9 +4,9 @@
 //   absorb_q  q~[b,h,c] = sum_d q_nope[b,h,d] W^UK_h[d,c]   ("Absorb key weights", first einsum)
 //   out_up    o[b,h,d]  = sum_c ctx[b,h,c]    W^UV_h[d,c]   ("Absorb key weights", last einsum)
 //
-// Both are a batch of 128 small GEMMs whose cost is reading W (8.4 MB per projection); each is run
-// "swap-AB" so that the 128 rows of one head's weight block are the MMA's M = 128 and the batch is
-// N (padded to a multiple of 16, at most 256 per CTA):
+// Both are a batch of 128 small GEMMs whose cost is reading W (8.4M bf16 weights, 16.8 MB, per
+// projection); each is run "swap-AB" so that the 128 rows of one head's weight block are the MMA's
+// M = 128 and the batch is N (padded to a multiple of 16, at most 256 per CTA):
 //   absorb_q: D[c, b] = W^UK_h^T[c, d] q_nope_h^T[d, b]   A = W^UK_h read MN-major, K = 128
 //   out_up:   D[d, b] = W^UV_h[d, c]   ctx_h^T[c, b]      A = W^UV_h read K-major,  K = 512
 // One CTA computes the tiles of one (head, batch block) and kMB 128-row blocks (two for absorb_q,
