@@ -46,6 +46,10 @@ SIGNATURES = {
                                         c_vp, c_i64, c_vp, c_i64,
                                         c_vp, c_i64, c_i64, c_vp, c_i64, c_i64,
                                         c_i32, c_vp, c_f32, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
+    "mla_decode_absorb_multi_topk": (c_i32, [MLADims, c_i32, c_i32, c_i32,
+                                             c_vp, c_i64, c_vp, c_i64,
+                                             c_vp, c_i64, c_i64, c_vp, c_i64, c_i64,
+                                             c_i32, c_vp, c_vp, c_i32, c_f32, c_vp, c_vp, c_vp, c_sz, c_vp, c_vp]),
     "mla_decode_absorb_static": (c_i32, [MLADims, c_i32, c_i32,
                                          c_vp, c_i64, c_vp, c_i64,
                                          c_vp, c_i64, c_i64, c_vp, c_i64, c_i64,

@@ -177,6 +177,39 @@ def mla_decode_absorb_multi(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_k
     return ctx
 
 
+def mla_decode_absorb_multi_topk(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_kv: torch.Tensor,
+                                 k_r: torch.Tensor, lengths: torch.Tensor, topk_idx: torch.Tensor, scale: float,
+                                 ctx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                                 workspace: Optional[torch.Tensor] = None, dev_err: Optional[torch.Tensor] = None,
+                                 stream=None) -> torch.Tensor:
+    """mla_decode_absorb_multi with a top-k set per new token: topk_idx int32 [B, T, k] (token s of
+    sequence b attends its set's rows t <= lengths[b] - T + s); returns ctx [B, T, n_h, d_c]."""
+    d = _dims(dims)
+    B, T = q_tilde.shape[0], q_tilde.shape[1]
+    n_max = c_kv.shape[1]
+    qt = q_tilde.reshape(B * T, d.n_h, -1)
+    qp = q_pe.reshape(B * T, d.n_h, -1)
+    ldqt, ldqp = _headrows(qt, "q_tilde"), _headrows(qp, "q_pe")
+    _rows(c_kv, "c_kv")
+    _rows(k_r, "k_r")
+    if lengths.dtype != torch.int32:
+        raise TypeError("lengths must be int32")
+    if topk_idx.dtype != torch.int32 or not topk_idx.is_contiguous() or tuple(topk_idx.shape[:2]) != (B, T):
+        raise TypeError("topk_idx must be a contiguous int32 [B, T, k] tensor")
+    k = topk_idx.shape[2]
+    if ctx is None:
+        ctx = torch.empty((B, T, d.n_h, d.d_c), dtype=q_tilde.dtype, device=q_tilde.device)
+    if workspace is None:
+        nbytes = mla_decode_workspace_size(d, q_tilde.dtype, B * T, n_max, k)
+        workspace = torch.empty((max(nbytes, 16),), dtype=torch.uint8, device=q_tilde.device)
+    check(lib().mla_decode_absorb_multi_topk(
+        d, _dt(q_tilde), B, T, _ptr(qt), ldqt, _ptr(qp), ldqp,
+        _ptr(c_kv), c_kv.stride(0), c_kv.stride(1), _ptr(k_r), k_r.stride(0), k_r.stride(1),
+        n_max, _ptr(lengths), _ptr(topk_idx), k, float(scale), _ptr(ctx), _ptr(lse), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(dev_err), _stream(stream)), "mla_decode_absorb_multi_topk")
+    return ctx
+
+
 def mla_decode_absorb_static(dims, q_tilde: torch.Tensor, q_pe: torch.Tensor, c_kv: torch.Tensor,
                              k_r: torch.Tensor, lengths: torch.Tensor, scale: float,
                              ctx: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,

@@ -282,6 +282,53 @@ mla_status mla_decode_absorb_multi(mla_dims dims, mla_dtype dtype, int32_t B, in
                      "mla_decode_absorb_multi launch");
 }
 
+mla_status mla_decode_absorb_multi_topk(mla_dims dims, mla_dtype dtype, int32_t B, int32_t T, const void* q_tilde,
+                                        int64_t ldqt, const void* q_pe, int64_t ldqp, const void* c_kv,
+                                        int64_t ckv_bstride, int64_t ckv_rstride, const void* k_r,
+                                        int64_t kr_bstride, int64_t kr_rstride, int32_t n_max,
+                                        const int32_t* lengths, const int32_t* topk_idx, int32_t topk, float scale,
+                                        void* ctx_out, float* lse_out, void* workspace, size_t ws_bytes,
+                                        int32_t* dev_err, void* stream) {
+  g_msg[0] = 0;
+  if (!topk_idx) return fail(MLA_ERR_INVALID_ARG, "NULL top-k index array");
+  if (T == 1)
+    return mla_decode_absorb(dims, dtype, B, q_tilde, ldqt, q_pe, ldqp, c_kv, ckv_bstride, ckv_rstride, k_r,
+                             kr_bstride, kr_rstride, n_max, lengths, topk_idx, topk, scale, ctx_out, lse_out,
+                             workspace, ws_bytes, dev_err, stream);
+  MLA_TRY(check_dims(dims, dtype));
+  if (B <= 0 || T < 1 || n_max <= 0 || T > n_max) return fail(MLA_ERR_INVALID_ARG, "need B > 0 and 1 <= T <= n_max");
+  if (topk < 1 || topk > n_max) return fail(MLA_ERR_INVALID_ARG, "topk must lie in [1, n_max]");
+  if ((int64_t)B * T * dims.n_h >= ((int64_t)1 << 31) || (int64_t)B * T > 65535)
+    return fail(MLA_ERR_UNSUPPORTED, "B * T query groups too many");
+  if (!q_tilde || !q_pe || !c_kv || !k_r || !lengths || !ctx_out) return fail(MLA_ERR_INVALID_ARG, "NULL pointer");
+  if (ldqt < dims.d_c || ldqp < dims.d_r) return fail(MLA_ERR_INVALID_ARG, "query row stride too small");
+  if (ckv_rstride < dims.d_c || kr_rstride < dims.d_r || ckv_bstride < 0 || kr_bstride < 0)
+    return fail(MLA_ERR_INVALID_ARG, "cache stride too small");
+  if (!(scale > 0.f) || scale != scale) return fail(MLA_ERR_INVALID_ARG, "scale must be positive");
+  MLA_TRY(check_bf16_ptr(dtype, q_tilde, "q_tilde"));
+  MLA_TRY(check_bf16_ptr(dtype, q_pe, "q_pe"));
+  MLA_TRY(check_bf16_ptr(dtype, c_kv, "c_kv"));
+  MLA_TRY(check_bf16_ptr(dtype, k_r, "k_r"));
+  MLA_TRY(check_bf16_ptr(dtype, ctx_out, "ctx_out"));
+  const int32_t BT = B * T;
+  const size_t need = mla_decode_workspace_size(dims, dtype, BT, n_max, topk);
+  if (!workspace || ws_bytes < need)
+    return fail(MLA_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need, workspace ? ws_bytes : (size_t)0);
+  if (!aligned16(workspace)) return fail(MLA_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+  mla::DecodeArgs a;
+  a.n_h = dims.n_h; a.d_c = dims.d_c; a.d_r = dims.d_r; a.B = BT; a.T = T; a.n_max = n_max;
+  a.topk = topk;
+  a.q_tilde = q_tilde; a.ldqt = ldqt; a.q_pe = q_pe; a.ldqp = ldqp;
+  a.c_kv = c_kv; a.ckv_b = ckv_bstride; a.ckv_r = ckv_rstride;
+  a.k_r = k_r; a.kr_b = kr_bstride; a.kr_r = kr_rstride;
+  a.lengths = lengths; a.topk_idx = topk_idx; a.scale = scale;
+  a.ctx = ctx_out; a.lse = lse_out; a.err = dev_err;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const cudaError_t e = dtype == MLA_BF16 ? mla::decode_simt_launch<__nv_bfloat16>(a, workspace, st)
+                                          : mla::decode_simt_launch<float>(a, workspace, st);
+  return cuda_status(e, "mla_decode_absorb_multi_topk launch");
+}
+
 mla_status mla_decode_absorb_static(mla_dims dims, mla_dtype dtype, int32_t B, const void* q_tilde, int64_t ldqt,
                                     const void* q_pe, int64_t ldqp, const void* c_kv, int64_t ckv_bstride,
                                     int64_t ckv_rstride, const void* k_r, int64_t kr_bstride, int64_t kr_rstride,

@@ -82,25 +82,32 @@ __global__ void out_up_simt(int n_h, int d_c, int d_h, int d_v, int B, const T* 
 }
 
 // ----------------------------------------------------------------------------------------
-// decode: one warp per (head, sequence, split); lanes own latent columns lane + 32 i
+// decode: one warp per (head, query group, split); lanes own latent columns lane + 32 i.
+// kMulti: several new tokens per sequence, each with its own top-k set: query group b is token
+// b % T of cache sequence b / T, and it sees the cached rows t <= length - T + (b % T) of its set
+// (the prefill's causal rule applied after the set, as in the sparse prefill).
 // ----------------------------------------------------------------------------------------
-template <typename T, int NC, int NR>
+template <typename T, int NC, int NR, bool kMulti>
 __global__ void decode_simt(DecodeArgs a, int n_splits, float* __restrict__ ws_o,
                             float2* __restrict__ ws_ml) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x * (blockDim.x >> 5) + warp;
   const int b = blockIdx.y, split = blockIdx.z;
   if (h >= a.n_h) return;
-  int len = a.lengths[b];
-  if (len < 1 || len > a.n_max) {
+  const int seq = kMulti ? b / a.T : b;  // cache sequence of this query group
+  int len = a.lengths[seq];
+  bool bad_len = false;
+  if (len < (kMulti ? a.T : 1) || len > a.n_max) {
     if (lane == 0 && h == 0 && split == 0) raise_error(a.err, MLA_ERR_LENGTH);
     len = len < 0 ? 0 : (len > a.n_max ? a.n_max : len);
+    bad_len = kMulti;  // several tokens: the sequence's tokens get ctx = 0 and lse = -inf
   }
+  const int last = kMulti ? len - a.T + b % a.T : len - 1;  // the last row this query sees
   const int n_keys_cap = a.topk_idx ? a.topk : a.n_max;
   const int n_keys = a.topk_idx ? a.topk : len;
   const int chunk = (n_keys_cap + n_splits - 1) / n_splits;
   const int j0 = split * chunk;
-  const int j1 = min(j0 + chunk, n_keys);
+  const int j1 = bad_len ? j0 : min(j0 + chunk, n_keys);
 
   const T* qt = static_cast<const T*>(a.q_tilde) + ((int64_t)b * a.n_h + h) * a.ldqt;
   const T* qp = static_cast<const T*>(a.q_pe) + ((int64_t)b * a.n_h + h) * a.ldqp;
@@ -116,8 +123,8 @@ __global__ void decode_simt(DecodeArgs a, int n_splits, float* __restrict__ ws_o
     const int r = lane + 32 * i;
     qr[i] = r < a.d_r ? to_f32(qp[r]) : 0.f;
   }
-  const T* cb = static_cast<const T*>(a.c_kv) + (int64_t)b * a.ckv_b;
-  const T* rb = static_cast<const T*>(a.k_r) + (int64_t)b * a.kr_b;
+  const T* cb = static_cast<const T*>(a.c_kv) + (int64_t)seq * a.ckv_b;
+  const T* rb = static_cast<const T*>(a.k_r) + (int64_t)seq * a.kr_b;
   float m = -INFINITY, l = 0.f;
   for (int j = j0; j < j1; ++j) {
     int t = j;
@@ -127,6 +134,7 @@ __global__ void decode_simt(DecodeArgs a, int n_splits, float* __restrict__ ws_o
         if (lane == 0 && h == 0) raise_error(a.err, MLA_ERR_INDEX);
         continue;
       }
+      if (kMulti && t > last) continue;  // a later new token's row: removed by the causal rule
     }
     const T* crow = cb + (int64_t)t * a.ckv_r;
     const T* rrow = rb + (int64_t)t * a.kr_r;
@@ -328,6 +336,17 @@ size_t decode_simt_workspace(int n_h, int d_c, int B, int n_keys_cap) {
   return (size_t)s * B * n_h * (d_c * sizeof(float) + sizeof(float2)) + 256;
 }
 
+template <typename T, bool kMulti>
+void decode_simt_dispatch(const DecodeArgs& a, dim3 grid, int splits, float* ws_o, float2* ws_ml, cudaStream_t st) {
+  if (a.d_c <= 64 && a.d_r <= 32)
+    decode_simt<T, 2, 1, kMulti><<<grid, 128, 0, st>>>(a, splits, ws_o, ws_ml);
+  else if (a.d_c <= 512 && a.d_r <= 64)
+    decode_simt<T, 16, 2, kMulti><<<grid, 128, 0, st>>>(a, splits, ws_o, ws_ml);
+  else
+    decode_simt<T, 32, 4, kMulti><<<grid, 128, 0, st>>>(a, splits, ws_o, ws_ml);
+}
+
+// a.B query groups; a.T > 1 (with a top-k set) is the several-token decode over a.B / a.T sequences
 template <typename T>
 cudaError_t decode_simt_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   const int n_keys_cap = a.topk_idx ? a.topk : a.n_max;
@@ -335,12 +354,10 @@ cudaError_t decode_simt_launch(const DecodeArgs& a, void* ws, cudaStream_t st) {
   float* ws_o = static_cast<float*>(ws);
   float2* ws_ml = reinterpret_cast<float2*>(ws_o + (size_t)splits * a.B * a.n_h * a.d_c);
   dim3 grid((a.n_h + 3) / 4, a.B, splits);
-  if (a.d_c <= 64 && a.d_r <= 32)
-    decode_simt<T, 2, 1><<<grid, 128, 0, st>>>(a, splits, ws_o, ws_ml);
-  else if (a.d_c <= 512 && a.d_r <= 64)
-    decode_simt<T, 16, 2><<<grid, 128, 0, st>>>(a, splits, ws_o, ws_ml);
+  if (a.T > 1 && a.topk_idx)
+    decode_simt_dispatch<T, true>(a, grid, splits, ws_o, ws_ml, st);
   else
-    decode_simt<T, 32, 4><<<grid, 128, 0, st>>>(a, splits, ws_o, ws_ml);
+    decode_simt_dispatch<T, false>(a, grid, splits, ws_o, ws_ml, st);
   cudaError_t e = launch_check();
   if (e != cudaSuccess || splits == 1) return e;
   combine_simt<T><<<dim3(a.n_h, a.B), 128, 0, st>>>(a, splits, ws_o, ws_ml);

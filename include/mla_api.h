@@ -193,8 +193,8 @@ mla_status mla_decode_absorb_fp8kv(mla_dims dims, int32_t B, const void* q_tilde
  *                                    sets MLA_ERR_LENGTH in dev_err and its tokens get ctx = 0,
  *                                    lse = -inf
  *   workspace                        mla_decode_workspace_size(dims, dtype, B * T, n_max, 0) bytes
- * bf16 DeepSeek dimensions only, no top-k set for T > 1 (MLA_ERR_UNSUPPORTED).  Each token runs as
- * its own query group over the shared cache rows of its sequence.  Asynchronous on `stream`.
+ * bf16 DeepSeek dimensions only; a top-k set per token is mla_decode_absorb_multi_topk.  Each token
+ * runs as its own query group over the shared cache rows of its sequence.  Asynchronous on `stream`.
  * Residency and MLA_DECODE_SLICED_MERGE as for mla_decode_absorb.
  */
 mla_status mla_decode_absorb_multi(mla_dims dims, mla_dtype dtype, int32_t B, int32_t T,
@@ -204,6 +204,32 @@ mla_status mla_decode_absorb_multi(mla_dims dims, mla_dtype dtype, int32_t B, in
                                    int32_t n_max, const int32_t* lengths, float scale, void* ctx_out,
                                    float* lse_out, void* workspace, size_t ws_bytes, int32_t* dev_err,
                                    void* stream);
+
+/*
+ * mla_decode_absorb_multi_topk - mla_decode_absorb_multi with a top-k set per new token (the V3.2
+ * decode excerpt's index mask, one set per query as in the sparse prefill, "Value up-projection",
+ * MHA-prefill excerpt, `index_mask += mask`): token s of sequence b attends the positions of its
+ * set that the causal rule keeps, t <= lengths[b] - T + s; later positions in a set are removed by
+ * that rule, not flagged.
+ *   topk_idx  DEVICE int32 [B, T, topk] contiguous (row b * T + s is token s of sequence b);
+ *             1 <= topk <= n_max; indices distinct per row (the set precondition of the gather
+ *             decode); an index outside [0, lengths[b]) sets MLA_ERR_INDEX and is skipped
+ *   lengths   DEVICE int32 [B] in [T, n_max]; another length sets MLA_ERR_LENGTH and the
+ *             sequence's tokens get ctx = 0, lse = -inf
+ *   workspace mla_decode_workspace_size(dims, dtype, B * T, n_max, topk) bytes
+ *   Other arguments as in mla_decode_absorb_multi; bf16 (DeepSeek dimensions) or fp32.  T = 1 is
+ *   mla_decode_absorb with topk_idx.  B * T <= 65535.
+ * For T > 1 the CUDA-core kernel runs (one warp per head and query, split over the set, with a
+ * merge pass when split): a query that selects no visible row gets ctx = 0 and lse = -inf.
+ * Asynchronous on `stream`.
+ */
+mla_status mla_decode_absorb_multi_topk(mla_dims dims, mla_dtype dtype, int32_t B, int32_t T,
+                                        const void* q_tilde, int64_t ldqt, const void* q_pe, int64_t ldqp,
+                                        const void* c_kv, int64_t ckv_bstride, int64_t ckv_rstride,
+                                        const void* k_r, int64_t kr_bstride, int64_t kr_rstride,
+                                        int32_t n_max, const int32_t* lengths, const int32_t* topk_idx,
+                                        int32_t topk, float scale, void* ctx_out, float* lse_out,
+                                        void* workspace, size_t ws_bytes, int32_t* dev_err, void* stream);
 
 /*
  * mla_decode_absorb_static - mla_decode_absorb for the bf16 dense decode (no top-k) WITHOUT a

@@ -135,8 +135,9 @@ def test_host_validation_codes(L):
 
 
 def test_host_validation_codes_newer_entry_points(L):
-    """The FP8-cache decode, the multi-token decode, the static-scratch decode and the wait self-test
-    refuse bad arguments on the host (before any launch)."""
+    """The FP8-cache decode, the multi-token decode (with and without per-token top-k sets), the
+    static-scratch decode and the wait self-test refuse bad arguments on the host (before any
+    launch)."""
     tiny = _capi.MLADims(4, 64, 16, 32, 32)
 
     def fp8(**kw):
@@ -192,6 +193,27 @@ def test_host_validation_codes_newer_entry_points(L):
     assert static(dt=_capi.MLA_F32) == 2
     assert static(B=0) == 1
     assert static(B=100_000, n_max=65536) == 6   # more split-KV scratch than the built-in array holds
+    def multi_topk(**kw):
+        a = dict(dims=DS, dt=_capi.MLA_BF16, B=2, T=2, qt=FAKE, ldqt=512, qp=FAKE, ldqp=64, ckv=FAKE,
+                 cb=4096 * 576, cr=576, kr=FAKE, kb=4096 * 576, krr=576, n_max=4096, lengths=FAKE, tk=FAKE,
+                 k=64, scale=0.07, ctx=FAKE, lse=None, ws=FAKE, wsb=1 << 40, err=None)
+        a.update(kw)
+        return L.mla_decode_absorb_multi_topk(*a.values(), None)
+
+    assert multi_topk(tk=None) == 1          # the sets are the point of this call
+    assert multi_topk(dims=tiny) == 2        # bf16 needs the DeepSeek dimensions
+    assert multi_topk(T=0) == 1
+    assert multi_topk(T=4097) == 1
+    assert multi_topk(k=0) == 1
+    assert multi_topk(k=4097) == 1           # more selected rows than cache rows
+    assert multi_topk(B=40000) == 2          # more query groups than one grid dimension holds
+    assert multi_topk(lengths=None) == 1
+    assert multi_topk(cr=500) == 1
+    assert multi_topk(scale=float("nan")) == 1
+    assert multi_topk(qt=FAKE + 2) == 1      # misaligned bf16 rows
+    assert multi_topk(ws=None) == 6
+    assert multi_topk(wsb=16) == 6
+    assert multi_topk(T=1, ws=None) == 6     # T = 1 is the one-token top-k decode
     assert L.mla_selftest_wait_timeout(1_000_000, None, None) == 1
     assert L.mla_selftest_wait_timeout(10, FAKE, None) == 1            # below 1 us
     assert L.mla_selftest_wait_timeout(2_000_000_000, FAKE, None) == 1  # above 1 s
